@@ -1,0 +1,228 @@
+"""Python binding of libcsa -- hybrid compressed attention (CSA / HCA) on B200.
+
+A thin ctypes layer over the C ABI declared in ``include/csa.h``: it checks
+dtypes, devices and contiguity of torch tensors, passes their device pointers
+and the current CUDA stream, and raises :class:`CsaError` on a non-zero
+return code.  Every step of the computation runs in the library's CUDA
+kernels; there is no Python or CPU fallback.  If ``libcsa.so`` has not been
+built, loading fails with an error that says so.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK = 0
+CSA_ERR_INVALID = -1
+CSA_ERR_UNSUPPORTED = -2
+CSA_ERR_CUDA = -3
+CSA_ERR_TIMEOUT = -4
+CSA_ERR_WORKSPACE = -5
+
+# every symbol declared in include/csa.h
+SYMBOLS = (
+    "csa_compress",
+    "csa_index_topk_workspace",
+    "csa_index_topk",
+    "csa_attend_workspace",
+    "csa_attend",
+    "hca_attend_workspace",
+    "hca_attend",
+    "csa_last_error",
+    "csa_sync_status",
+    "csa_version",
+    "csa_launch_count",
+)
+
+
+class CsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libcsa error {code}: {msg}")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    """Mirror of ``csa_dims`` in include/csa.h."""
+
+    _fields_ = [
+        ("B", ctypes.c_int32), ("Tq", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("D", ctypes.c_int32), ("HI", ctypes.c_int32), ("dI", ctypes.c_int32),
+        ("K", ctypes.c_int32), ("W", ctypes.c_int32), ("m", ctypes.c_int32),
+        ("n_entries", ctypes.c_int32), ("entry_cap", ctypes.c_int64),
+        ("win_cap", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+    ]
+
+    def __init__(self, B=1, Tq=1, H=1, D=512, HI=4, dI=64, K=512, W=128, m=4, n_entries=0,
+                 entry_cap=None, win_cap=None, softmax_scale=1.0):
+        super().__init__(B, Tq, H, D, HI, dI, K, W, m, n_entries,
+                         n_entries if entry_cap is None else entry_cap,
+                         W if win_cap is None else win_cap, softmax_scale)
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcsa.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libcsa.so not built at {LIB_PATH}: run "
+                          "`python -m compressed_sparse_attention_16_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.csa_compress.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _I64, _I64, _I32, _P, _P]
+    L.csa_compress.restype = ctypes.c_int
+    L.csa_index_topk_workspace.argtypes = [ctypes.POINTER(Dims)]
+    L.csa_index_topk_workspace.restype = _SZ
+    L.csa_index_topk.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
+    L.csa_index_topk.restype = ctypes.c_int
+    for name in ("csa_attend_workspace", "hca_attend_workspace"):
+        getattr(L, name).argtypes = [ctypes.POINTER(Dims)]
+        getattr(L, name).restype = _SZ
+    L.csa_attend.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
+    L.csa_attend.restype = ctypes.c_int
+    L.hca_attend.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
+    L.hca_attend.restype = ctypes.c_int
+    L.csa_last_error.argtypes = []
+    L.csa_last_error.restype = ctypes.c_char_p
+    L.csa_sync_status.argtypes = [_P]
+    L.csa_sync_status.restype = ctypes.c_int
+    L.csa_version.argtypes = []
+    L.csa_version.restype = ctypes.c_int
+    L.csa_launch_count.argtypes = []
+    L.csa_launch_count.restype = ctypes.c_uint64
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != CSA_OK:
+        raise CsaError(rc, lib().csa_last_error().decode(errors="replace"))
+
+
+def _ptr(t: torch.Tensor | None, dtype, name: str, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+# ---------------------------------------------------------------------------
+# operations
+# ---------------------------------------------------------------------------
+
+
+def compress(x: torch.Tensor, z: torch.Tensor, m: int, codes: torch.Tensor, scales: torch.Tensor,
+             dst_first: int = 0, ring_cap: int = 0, pooled: torch.Tensor | None = None,
+             T: int | None = None, stream=None) -> None:
+    """csa_compress: pool full m-token blocks of x, z [B, Ttot, D] (first T tokens)
+    into codes u8 [B, cap, D] / scales f32 [B, cap] at slots dst_first + i."""
+    if x.dim() != 3 or z.shape != x.shape:
+        raise ValueError("x and z must be [B, T, D] of equal shape")
+    B, Ttot, D = x.shape
+    T = Ttot if T is None else T
+    if codes.dim() != 3 or codes.shape[0] != B or codes.shape[2] != D or scales.shape != codes.shape[:2]:
+        raise ValueError("codes must be [B, cap, D] and scales [B, cap]")
+    dev = x.device
+    _check(lib().csa_compress(_ptr(x, torch.float32, "x"), _ptr(z, torch.float32, "z", dev),
+                              B, T, D, m, Ttot * D,
+                              _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
+                              dst_first, codes.shape[1], ring_cap,
+                              _ptr(pooled, torch.float32, "pooled", dev), _stream(stream)))
+
+
+def index_topk_workspace(dims: Dims) -> int:
+    return int(lib().csa_index_topk_workspace(ctypes.byref(dims)))
+
+
+def attend_workspace(dims: Dims, dense: bool = False) -> int:
+    fn = lib().hca_attend_workspace if dense else lib().csa_attend_workspace
+    return int(fn(ctypes.byref(dims)))
+
+
+def _ws(workspace, nbytes, device):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        raise ValueError(f"this call needs a workspace of {nbytes} bytes")
+    return _ptr(workspace, torch.uint8, "workspace", device), workspace.numel()
+
+
+def index_topk(qI, w, kI, q_pos, dims: Dims, idx_out, score_out=None, workspace=None, stream=None):
+    """csa_index_topk: indexer scores + top-k; see include/csa.h."""
+    dev = qI.device
+    need = index_topk_workspace(dims)
+    wp, wn = _ws(workspace, need, dev)
+    _check(lib().csa_index_topk(_ptr(qI, torch.uint8, "qI"), _ptr(w, torch.float32, "w", dev),
+                                _ptr(kI, torch.uint8, "kI", dev), _ptr(q_pos, torch.int32, "q_pos", dev),
+                                ctypes.byref(dims), _ptr(idx_out, torch.int32, "idx_out", dev),
+                                _ptr(score_out, torch.float32, "score_out", dev), wp, wn, _stream(stream)))
+
+
+def attend(q, codes, scales, idx, win_codes, win_scales, q_pos, dims: Dims, out, lse=None,
+           workspace=None, stream=None):
+    """csa_attend: sparse shared-KV MQA over selected entries + window."""
+    dev = q.device
+    wp, wn = _ws(workspace, attend_workspace(dims, False), dev)
+    _check(lib().csa_attend(_ptr(q, torch.bfloat16, "q"), _ptr(codes, torch.uint8, "codes", dev),
+                            _ptr(scales, torch.float32, "scales", dev), _ptr(idx, torch.int32, "idx", dev),
+                            _ptr(win_codes, torch.uint8, "win_codes", dev),
+                            _ptr(win_scales, torch.float32, "win_scales", dev),
+                            _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
+                            _ptr(out, torch.bfloat16, "out", dev), _ptr(lse, torch.float32, "lse", dev),
+                            wp, wn, _stream(stream)))
+
+
+def hca_attend(q, codes, scales, win_codes, win_scales, q_pos, dims: Dims, out, lse=None,
+               workspace=None, stream=None):
+    """hca_attend: dense attention over every visible entry + window."""
+    dev = q.device
+    wp, wn = _ws(workspace, attend_workspace(dims, True), dev)
+    _check(lib().hca_attend(_ptr(q, torch.bfloat16, "q"), _ptr(codes, torch.uint8, "codes", dev),
+                            _ptr(scales, torch.float32, "scales", dev),
+                            _ptr(win_codes, torch.uint8, "win_codes", dev),
+                            _ptr(win_scales, torch.float32, "win_scales", dev),
+                            _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
+                            _ptr(out, torch.bfloat16, "out", dev), _ptr(lse, torch.float32, "lse", dev),
+                            wp, wn, _stream(stream)))
+
+
+def sync_status(stream=None) -> None:
+    """Wait for the stream and raise if a kernel flagged bad data or a timeout."""
+    _check(lib().csa_sync_status(_stream(stream)))
+
+
+def version() -> int:
+    return int(lib().csa_version())
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(lib().csa_launch_count())

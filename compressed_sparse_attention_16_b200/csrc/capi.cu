@@ -1,0 +1,229 @@
+// C ABI of libcsa: argument validation, error reporting, the device status
+// word, and dispatch to the kernels.  See include/csa.h for the contract of
+// every entry point.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace csa {
+
+int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
+                    uint8_t *codes, float *scales, int64_t dst_first, int64_t dst_bstride,
+                    int ring_cap, float *pooled, cudaStream_t stream);
+size_t index_topk_workspace(const csa_dims *d);
+int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+                      const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
+                      cudaStream_t stream);
+int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
+                  const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
+                  const csa_dims *d, uint16_t *out, float *lse, void *workspace, size_t ws_bytes,
+                  cudaStream_t stream);
+size_t attend_workspace(const csa_dims *d, bool dense);
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+static thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int check_launch(const char *what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return CSA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// device status word: one per device that loads the library
+// ---------------------------------------------------------------------------
+static __device__ unsigned g_status_word;
+
+unsigned *status_word_device_ptr() {
+  static std::mutex mu;
+  static unsigned *ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned *>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace csa
+
+using namespace csa;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int need_status() {
+  if (!status_word_device_ptr())
+    return fail(CSA_ERR_CUDA, "cannot resolve the device status word (no CUDA device?)");
+  return CSA_OK;
+}
+
+int check_attend_dims(const char *fn, const csa_dims *d, bool dense) {
+  if (!d) return fail(CSA_ERR_INVALID, "%s: dims is NULL", fn);
+  if (d->B < 0 || d->Tq < 0 || d->H < 1 || d->W < 1 || d->m < 1 || d->n_entries < 0)
+    return fail(CSA_ERR_INVALID, "%s: bad dims (B=%d Tq=%d H=%d W=%d m=%d n_entries=%d)", fn, d->B,
+                d->Tq, d->H, d->W, d->m, d->n_entries);
+  if (d->entry_cap < d->n_entries) return fail(CSA_ERR_INVALID, "%s: entry_cap < n_entries", fn);
+  if (d->win_cap < d->W) return fail(CSA_ERR_INVALID, "%s: win_cap (%d) < W (%d)", fn, d->win_cap, d->W);
+  if (d->D != 64 && d->D != 128 && d->D != 256 && d->D != 512)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: D=%d (supported 64, 128, 256, 512)", fn, d->D);
+  if (!dense && (d->K < 1 || d->K > 2048))
+    return fail(CSA_ERR_UNSUPPORTED, "%s: K=%d (supported 1..2048)", fn, d->K);
+  if (!(d->softmax_scale == d->softmax_scale)) return fail(CSA_ERR_INVALID, "%s: softmax_scale is NaN", fn);
+  return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_version(void) { return 100; }
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *csa_last_error(void) { return g_err; }
+
+int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D, int32_t m,
+                 int64_t x_batch_stride, uint8_t *codes, float *scales, int64_t dst_first,
+                 int64_t dst_batch_stride, int32_t ring_cap, float *pooled,
+                 csa_stream_t stream) {
+  clear_error();
+  if (B < 0 || T < 0 || m < 1) return fail(CSA_ERR_INVALID, "csa_compress: bad B/T/m (%d/%d/%d)", B, T, m);
+  if (D < 4 || D > 1024 || D % 4 || !pow2(D / 4))
+    return fail(CSA_ERR_UNSUPPORTED, "csa_compress: D=%d (needs D/4 a power of two, 4..1024)", D);
+  if (B == 0 || T < m) return CSA_OK;
+  if (!x || !z || !codes || !scales) return fail(CSA_ERR_INVALID, "csa_compress: NULL buffer");
+  if (!aligned16(x) || !aligned16(z) || (pooled && !aligned16(pooled)) || ((uintptr_t)codes & 3))
+    return fail(CSA_ERR_INVALID, "csa_compress: misaligned buffer");
+  if (x_batch_stride % 4 || (B > 1 && x_batch_stride < (int64_t)T * D))
+    return fail(CSA_ERR_INVALID, "csa_compress: x_batch_stride must be a multiple of 4 and >= T*D");
+  if (dst_first < 0 || ring_cap < 0) return fail(CSA_ERR_INVALID, "csa_compress: negative dst_first/ring_cap");
+  if (ring_cap == 0 && B > 1 && dst_batch_stride < dst_first + T / m)
+    return fail(CSA_ERR_INVALID, "csa_compress: dst_batch_stride too small");
+  if (ring_cap > 0 && B > 1 && dst_batch_stride < ring_cap)
+    return fail(CSA_ERR_INVALID, "csa_compress: dst_batch_stride < ring_cap");
+  return launch_compress(x, z, B, T, D, m, x_batch_stride, codes, scales, dst_first,
+                         dst_batch_stride, ring_cap, pooled, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t csa_index_topk_workspace(const csa_dims *d) {
+  if (!d || d->B < 0 || d->Tq < 0 || d->n_entries < 0) return 0;
+  return index_topk_workspace(d);
+}
+
+int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+                   const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
+                   size_t workspace_bytes, csa_stream_t stream) {
+  clear_error();
+  if (!d) return fail(CSA_ERR_INVALID, "csa_index_topk: dims is NULL");
+  if (d->B < 0 || d->Tq < 0 || d->m < 1 || d->n_entries < 0 || d->entry_cap < d->n_entries)
+    return fail(CSA_ERR_INVALID, "csa_index_topk: bad dims");
+  if (d->K < 1 || d->K > 2048) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: K=%d (1..2048)", d->K);
+  if ((d->dI != 32 && d->dI != 64) || d->HI < 1 || d->HI > 8)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d dI=%d", d->HI, d->dI);
+  if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
+  if (!qI || !w || !kI || !q_pos || !idx_out) return fail(CSA_ERR_INVALID, "csa_index_topk: NULL buffer");
+  if (!aligned16(kI) || ((uintptr_t)qI & 3) || ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) ||
+      ((uintptr_t)idx_out & 3) || ((uintptr_t)score_out & 3))
+    return fail(CSA_ERR_INVALID, "csa_index_topk: misaligned buffer");
+  const size_t need = index_topk_workspace(d);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace needs %zu bytes (got %zu)", need,
+                workspace_bytes);
+  if (int rc = need_status()) return rc;
+  return launch_index_topk(qI, w, kI, q_pos, d, idx_out, score_out, workspace,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t csa_attend_workspace(const csa_dims *d) { return d ? attend_workspace(d, false) : 0; }
+size_t hca_attend_workspace(const csa_dims *d) { return d ? attend_workspace(d, true) : 0; }
+
+static int attend_common(const char *fn, const uint16_t *q, const uint8_t *codes,
+                         const float *scales, const int32_t *idx, const uint8_t *win_codes,
+                         const float *win_scales, const int32_t *q_pos, const csa_dims *d,
+                         uint16_t *out, float *lse, void *workspace, size_t workspace_bytes,
+                         csa_stream_t stream) {
+  clear_error();
+  const bool dense = idx == nullptr;
+  if (int rc = check_attend_dims(fn, d, dense)) return rc;
+  if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
+  if (!q || !win_codes || !win_scales || !q_pos || !out || (d->n_entries > 0 && (!codes || !scales)))
+    return fail(CSA_ERR_INVALID, "%s: NULL buffer", fn);
+  if (!aligned16(q) || !aligned16(out) || (codes && !aligned16(codes)) || !aligned16(win_codes) ||
+      ((uintptr_t)q_pos & 3) || ((uintptr_t)idx & 3) || ((uintptr_t)lse & 3) ||
+      ((uintptr_t)scales & 3) || ((uintptr_t)win_scales & 3))
+    return fail(CSA_ERR_INVALID, "%s: misaligned buffer", fn);
+  const size_t need = attend_workspace(d, dense);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(CSA_ERR_WORKSPACE, "%s: workspace needs %zu bytes (got %zu)", fn, need, workspace_bytes);
+  if (int rc = need_status()) return rc;
+  return launch_attend(q, codes, scales, idx, win_codes, win_scales, q_pos, d, out, lse, workspace,
+                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int csa_attend(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
+               const uint8_t *win_codes, const float *win_scales, const int32_t *q_pos,
+               const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+               size_t workspace_bytes, csa_stream_t stream) {
+  if (!idx) {
+    clear_error();
+    return fail(CSA_ERR_INVALID, "csa_attend: idx is NULL (use hca_attend for dense attention)");
+  }
+  return attend_common("csa_attend", q, codes, scales, idx, win_codes, win_scales, q_pos, d, out,
+                       lse, workspace, workspace_bytes, stream);
+}
+
+int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
+               const uint8_t *win_codes, const float *win_scales, const int32_t *q_pos,
+               const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+               size_t workspace_bytes, csa_stream_t stream) {
+  return attend_common("hca_attend", q, codes, scales, nullptr, win_codes, win_scales, q_pos, d,
+                       out, lse, workspace, workspace_bytes, stream);
+}
+
+int csa_sync_status(csa_stream_t stream) {
+  clear_error();
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_sync_status: %s", cudaGetErrorString(e));
+  unsigned *p = status_word_device_ptr();
+  if (!p) return fail(CSA_ERR_CUDA, "csa_sync_status: no device status word");
+  unsigned v = 0;
+  e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(unsigned));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_sync_status: %s", cudaGetErrorString(e));
+  if (v & STATUS_TIMEOUT) return fail(CSA_ERR_TIMEOUT, "a device-side wait timed out (status 0x%x)", v);
+  if (v & (STATUS_BAD_WEIGHT | STATUS_BAD_INDEX | STATUS_BAD_POSITION))
+    return fail(CSA_ERR_INVALID, "invalid device data: %s%s%s (status 0x%x)",
+                (v & STATUS_BAD_WEIGHT) ? "indexer weight off the 1/16 grid; " : "",
+                (v & STATUS_BAD_INDEX) ? "attention index out of range; " : "",
+                (v & STATUS_BAD_POSITION) ? "negative query position" : "", v);
+  return CSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Shared device helpers and host error plumbing for libcsa.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "csa.h"
+
+namespace csa {
+
+// ---------------------------------------------------------------------------
+// host side: thread-local error message
+// ---------------------------------------------------------------------------
+int fail(int code, const char *fmt, ...);
+int check_launch(const char *what);
+void count_launches(unsigned n);   // bookkeeping for csa_launch_count()
+void clear_error();
+
+// ---------------------------------------------------------------------------
+// device status word (set by kernels, read + cleared by csa_sync_status)
+// ---------------------------------------------------------------------------
+enum : unsigned {
+  STATUS_TIMEOUT = 1u,      // a bounded wait gave up
+  STATUS_BAD_WEIGHT = 2u,   // indexer weight not a multiple of 1/16 in [0, 1]
+  STATUS_BAD_INDEX = 4u,    // attention index outside [0, n_entries) other than -1
+  STATUS_BAD_POSITION = 8u, // negative query position (treated as position 0 / no entries)
+};
+unsigned *status_word_device_ptr();   // address of the status word, current device
+
+__device__ __forceinline__ void raise_status(unsigned *status, unsigned bit) {
+  atomicOr(status, bit);
+}
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Two E4M3 codes (low byte first) -> two floats (exact).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t two) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+  return __half22float2(*reinterpret_cast<__half2 *>(&h));
+}
+
+// PTX prmt in its default mode: each selector nibble picks one of the 8 bytes
+// of {b:a}; if the nibble's bit 3 is set, the picked byte's sign bit is
+// replicated instead of copying it.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+}  // namespace csa

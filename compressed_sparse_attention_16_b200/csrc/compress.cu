@@ -1,0 +1,142 @@
+// Softmax-gated pooling of m-token blocks into FP8-E4M3 entries with a
+// per-entry fp32 scale.
+//
+// Page: "DeepSeek V4 Flash：知っておくべき284Bパラメータのオープンソースモデル"
+// (studioglobal.ai), section "アテンションのブレイクスルー：CSAとHCA" --
+// softmax-gated pooling compresses the KV entries along the sequence; page
+// "DeepSeek V4とOpenCode" (hazakura.dev), section "衝撃1：CSA + HCA" -- m = 4
+// for CSA, m' = 128 for HCA; page "DeepSeek V4 1M context window agent
+// efficient inference" (ai-papers.net), section "ハイブリッドアテンションの
+// 仕組み" -- KV entries stored in FP8.
+//
+// The op is HBM-bound: 8 bytes read per (token, channel), 1/m byte written.
+// One group of D/4 threads owns one entry; each thread owns 4 channels and
+// streams the block's tokens with 16-byte loads, keeping a per-channel online
+// softmax (running max, normaliser and weighted sum).  The group then reduces
+// the entry's amax, and every thread quantises its 4 channels and stores them
+// as one 32-bit word.
+#include "common.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+struct OnlineSoftmax4 {
+  float mx[4], l[4], acc[4];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) { mx[c] = -INFINITY; l[c] = 0.f; acc[c] = 0.f; }
+  }
+  __device__ __forceinline__ void push(const float4 &xv, const float4 &zv) {
+    const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+    const float zs[4] = {zv.x, zv.y, zv.z, zv.w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (zs[c] > mx[c]) {
+        const float r = expf(mx[c] - zs[c]);     // 0 on the first token
+        l[c] = fmaf(l[c], r, 1.f);
+        acc[c] = fmaf(acc[c], r, xs[c]);
+        mx[c] = zs[c];
+      } else {
+        const float p = expf(zs[c] - mx[c]);
+        l[c] += p;
+        acc[c] = fmaf(p, xs[c], acc[c]);
+      }
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads)
+compress_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_per_seq,
+                int64_t n_total, int D, int m, int64_t x_bstride, uint8_t *__restrict__ codes,
+                float *__restrict__ scales, int64_t dst_first, int64_t dst_bstride, int ring_cap,
+                float *__restrict__ pooled) {
+  __shared__ float red[kThreads / 32];
+  const int L = D >> 2;                       // threads per entry
+  const int groups = kThreads / L;            // entries per CTA (L divides 256 or L >= 256 handled by host)
+  const int g = threadIdx.x / L;
+  const int lane = threadIdx.x - g * L;
+  const int64_t e = (int64_t)blockIdx.x * groups + g;
+  const bool active = (g < groups) && (e < n_total);
+
+  float C[4] = {0.f, 0.f, 0.f, 0.f};
+  int64_t b = 0, i = 0;
+  if (active) {
+    b = e / n_per_seq;
+    i = e - b * n_per_seq;
+    const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + lane;
+    const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + lane;
+    OnlineSoftmax4 sm;
+    sm.init();
+    int j = 0;
+    for (; j + kUnroll <= m; j += kUnroll) {
+      float4 xv[kUnroll], zv[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        xv[u] = __ldg(xp + (int64_t)(j + u) * L);
+        zv[u] = __ldg(zp + (int64_t)(j + u) * L);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) sm.push(xv[u], zv[u]);
+    }
+    for (; j < m; ++j) sm.push(__ldg(xp + (int64_t)j * L), __ldg(zp + (int64_t)j * L));
+#pragma unroll
+    for (int c = 0; c < 4; ++c) C[c] = __fdiv_rn(sm.acc[c], sm.l[c]);
+  }
+
+  // amax over the entry's L threads
+  float a = fmaxf(fmaxf(fabsf(C[0]), fabsf(C[1])), fmaxf(fabsf(C[2]), fabsf(C[3])));
+  const int width = L < 32 ? L : 32;
+  for (int o = width >> 1; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (L > 32) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = a;
+    __syncthreads();
+    const int w0 = (g * L) >> 5, nw = L >> 5;
+    a = 0.f;
+    for (int k = 0; k < nw; ++k) a = fmaxf(a, red[w0 + k]);
+  }
+  if (!active) return;
+
+  float s = __fdiv_rn(a, 448.f);
+  if (!(s > 0.f)) s = 1.f;
+  uint32_t word = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float r = __fdiv_rn(C[c], s);
+    const uint32_t q = __nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+    word |= q << (8 * c);
+  }
+  int64_t slot = dst_first + i;
+  if (ring_cap > 0) slot %= ring_cap;
+  const int64_t ent = b * dst_bstride + slot;
+  reinterpret_cast<uint32_t *>(codes + ent * D)[lane] = word;
+  if (lane == 0) scales[ent] = s;
+  if (pooled) {
+    reinterpret_cast<float4 *>(pooled + (b * n_per_seq + i) * (int64_t)D)[lane] =
+        make_float4(C[0], C[1], C[2], C[3]);
+  }
+}
+
+}  // namespace
+
+int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
+                    uint8_t *codes, float *scales, int64_t dst_first, int64_t dst_bstride,
+                    int ring_cap, float *pooled, cudaStream_t stream) {
+  const int n = T / m;
+  const int64_t total = (int64_t)B * n;
+  if (total == 0) return CSA_OK;
+  const int L = D / 4;
+  const int groups = kThreads / L;
+  const int64_t grid = (total + groups - 1) / groups;
+  if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
+  compress_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(x, z, n, total, D, m, x_bstride, codes,
+                                                           scales, dst_first, dst_bstride, ring_cap,
+                                                           pooled);
+  count_launches(1);
+  return check_launch("compress_kernel");
+}
+
+}  // namespace csa

@@ -1,0 +1,168 @@
+"""Host orchestration of the hybrid-attention path over the C ABI.
+
+Nothing here computes: each function allocates caller-side buffers with
+torch (device memory) and sequences the library's asynchronous calls on the
+current CUDA stream.
+
+* :func:`prefill` -- CSA over a whole sequence: pool every m-token block into
+  the FP8 cache, store every token as a window entry, run the indexer + top-k
+  for every position and attend.
+* :class:`DecodeState` -- a decode-time cache (compressed entries, indexer
+  keys, a window ring of ``win_cap`` tokens) that grows by one compressed
+  entry per ``m`` appended tokens, with :meth:`DecodeState.step` running one
+  append + query step (CSA: index, top-k, attend; HCA: dense attend).
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+from . import Dims, attend, attend_workspace, compress, hca_attend, index_topk, index_topk_workspace
+
+
+def _ws(nbytes: int, device) -> torch.Tensor | None:
+    return torch.empty(nbytes, dtype=torch.uint8, device=device) if nbytes else None
+
+
+@dataclasses.dataclass
+class PrefillResult:
+    out: torch.Tensor        # bf16 [B, T, H, D]
+    lse: torch.Tensor        # f32 [B, T, H]
+    idx: torch.Tensor        # int32 [B, T, K]
+    score: torch.Tensor      # f32 [B, T, K]
+    codes: torch.Tensor      # u8 [B, N, D]
+    scales: torch.Tensor     # f32 [B, N]
+    win_codes: torch.Tensor  # u8 [B, T, D]
+    win_scales: torch.Tensor  # f32 [B, T]
+
+
+def prefill(x, z, q, qI, w, kI, *, m: int, K: int, W: int, softmax_scale: float = 1.0,
+            pooled: torch.Tensor | None = None) -> PrefillResult:
+    """CSA prefill: every position 0..T-1 of each sequence is a query.
+
+    x, z: f32 [B, T, D]; q: bf16 [B, T, H, D]; qI: u8 [B, T, HI, dI/2];
+    w: f32 [B, T, HI]; kI: u8 [B, T // m, dI/2].
+    """
+    B, T, D = x.shape
+    H = q.shape[2]
+    HI, dI = qI.shape[2], 2 * qI.shape[3]
+    dev = x.device
+    N = T // m
+    codes = torch.empty((B, N, D), dtype=torch.uint8, device=dev)
+    scales = torch.empty((B, N), dtype=torch.float32, device=dev)
+    win_codes = torch.empty((B, T, D), dtype=torch.uint8, device=dev)
+    win_scales = torch.empty((B, T), dtype=torch.float32, device=dev)
+    compress(x, z, m, codes, scales, pooled=pooled)
+    compress(x, z, 1, win_codes, win_scales)
+    q_pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    dims = Dims(B=B, Tq=T, H=H, D=D, HI=HI, dI=dI, K=K, W=W, m=m, n_entries=N, entry_cap=N,
+                win_cap=T, softmax_scale=softmax_scale)
+    idx = torch.empty((B, T, K), dtype=torch.int32, device=dev)
+    score = torch.empty((B, T, K), dtype=torch.float32, device=dev)
+    index_topk(qI, w, kI, q_pos, dims, idx, score, workspace=_ws(index_topk_workspace(dims), dev))
+    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, T, H), dtype=torch.float32, device=dev)
+    attend(q, codes, scales, idx, win_codes, win_scales, q_pos, dims, out, lse,
+           workspace=_ws(attend_workspace(dims), dev))
+    return PrefillResult(out, lse, idx, score, codes, scales, win_codes, win_scales)
+
+
+class DecodeState:
+    """Decode cache for B sequences: compressed entries, indexer keys and a
+    window ring.  Capacity is fixed at construction (``entry_cap`` entries).
+
+    ``dense=True`` makes it an HCA cache (no indexer, dense attention).
+    """
+
+    def __init__(self, B: int, D: int, H: int, m: int, W: int, entry_cap: int, *, K: int = 512,
+                 HI: int = 4, dI: int = 64, win_cap: int | None = None, dense: bool = False,
+                 softmax_scale: float = 1.0, device="cuda"):
+        self.B, self.D, self.H, self.m, self.W, self.K = B, D, H, m, W, K
+        self.HI, self.dI, self.dense = HI, dI, dense
+        self.win_cap = W if win_cap is None else win_cap
+        self.entry_cap = entry_cap
+        self.softmax_scale = softmax_scale
+        self.device = torch.device(device)
+        dev = self.device
+        self.codes = torch.zeros((B, entry_cap, D), dtype=torch.uint8, device=dev)
+        self.scales = torch.ones((B, entry_cap), dtype=torch.float32, device=dev)
+        self.win_codes = torch.zeros((B, self.win_cap, D), dtype=torch.uint8, device=dev)
+        self.win_scales = torch.ones((B, self.win_cap), dtype=torch.float32, device=dev)
+        self.kI = None if dense else torch.zeros((B, entry_cap, dI // 2), dtype=torch.uint8, device=dev)
+        self.n_tokens = 0
+        self.q_pos = torch.zeros((B, 1), dtype=torch.int32, device=dev)
+        self.idx = None if dense else torch.empty((B, 1, K), dtype=torch.int32, device=dev)
+        self.score = None if dense else torch.empty((B, 1, K), dtype=torch.float32, device=dev)
+        self.out = torch.empty((B, 1, H, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, 1, H), dtype=torch.float32, device=dev)
+        self._ws_index = None
+        self._ws_attend = None
+
+    @property
+    def n_entries(self) -> int:
+        return self.n_tokens // self.m
+
+    def dims(self) -> Dims:
+        return Dims(B=self.B, Tq=1, H=self.H, D=self.D, HI=self.HI, dI=self.dI, K=self.K, W=self.W,
+                    m=self.m, n_entries=self.n_entries, entry_cap=self.entry_cap,
+                    win_cap=self.win_cap, softmax_scale=self.softmax_scale)
+
+    def prefill_context(self, x: torch.Tensor, z: torch.Tensor, T: int, kI: torch.Tensor | None = None):
+        """Compress tokens [0, T) of x, z [B, >=T, D] into the cache (setup).
+
+        kI (u8 [B, >= T//m, dI/2]) gives the indexer keys of those entries.
+        """
+        assert self.n_tokens == 0 and T // self.m <= self.entry_cap
+        compress(x, z, self.m, self.codes, self.scales, T=T)
+        lo = max(0, T - self.win_cap)
+        if T > lo:
+            compress(x[:, lo:T].contiguous(), z[:, lo:T].contiguous(), 1, self.win_codes,
+                     self.win_scales, dst_first=lo, ring_cap=self.win_cap)
+        if kI is not None and self.kI is not None:
+            self.kI[:, : T // self.m].copy_(kI[:, : T // self.m])
+        self.n_tokens = T
+
+    def append(self, x_new: torch.Tensor, z_new: torch.Tensor, kI_new: torch.Tensor | None = None):
+        """Append n tokens (x_new, z_new: f32 [B, n, D], n a multiple of m when the
+        cache is block aligned): completed blocks become entries, every token
+        enters the window ring.  kI_new (u8 [B, n//m, dI/2]) are the new
+        entries' indexer keys."""
+        n = x_new.shape[1]
+        assert self.n_tokens % self.m == 0 and n % self.m == 0
+        first = self.n_entries
+        assert first + n // self.m <= self.entry_cap
+        compress(x_new, z_new, self.m, self.codes, self.scales, dst_first=first)
+        compress(x_new, z_new, 1, self.win_codes, self.win_scales, dst_first=self.n_tokens,
+                 ring_cap=self.win_cap)
+        if kI_new is not None and self.kI is not None:
+            self.kI[:, first:first + n // self.m].copy_(kI_new)
+        self.n_tokens += n
+
+    def query(self, q: torch.Tensor, qI: torch.Tensor | None = None, w: torch.Tensor | None = None):
+        """One query per sequence at position n_tokens - 1.  q: bf16 [B, 1, H, D];
+        qI: u8 [B, 1, HI, dI/2], w: f32 [B, 1, HI] (CSA only)."""
+        self.q_pos.fill_(self.n_tokens - 1)
+        d = self.dims()
+        if self.dense:
+            nb = attend_workspace(d, True)
+            if nb and (self._ws_attend is None or self._ws_attend.numel() < nb):
+                self._ws_attend = _ws(nb, self.device)
+            hca_attend(q, self.codes, self.scales, self.win_codes, self.win_scales, self.q_pos, d,
+                       self.out, self.lse, workspace=self._ws_attend)
+            return self.out, self.lse
+        nb = index_topk_workspace(d)
+        if nb and (self._ws_index is None or self._ws_index.numel() < nb):
+            self._ws_index = _ws(nb, self.device)
+        index_topk(qI, w, self.kI, self.q_pos, d, self.idx, self.score, workspace=self._ws_index)
+        nb = attend_workspace(d, False)
+        if nb and (self._ws_attend is None or self._ws_attend.numel() < nb):
+            self._ws_attend = _ws(nb, self.device)
+        attend(q, self.codes, self.scales, self.idx, self.win_codes, self.win_scales, self.q_pos, d,
+               self.out, self.lse, workspace=self._ws_attend)
+        return self.out, self.lse
+
+    def step(self, x_new, z_new, q, qI=None, w=None, kI_new=None):
+        """Append tokens then run one query per sequence at the newest position."""
+        self.append(x_new, z_new, kI_new)
+        return self.query(q, qI, w)

@@ -1,0 +1,206 @@
+/*
+ * csa.h -- C ABI of the B200 hybrid compressed-attention library (libcsa.so).
+ *
+ * The library implements the data-parallel path of DeepSeek-V4-style hybrid
+ * attention as four asynchronous GPU operations:
+ *
+ *   csa_compress    softmax-gated pooling of m-token blocks into FP8 entries
+ *   csa_index_topk  FP4 Lightning-Indexer scores + per-query top-k selection
+ *   csa_attend      shared-KV multi-query attention over selected entries and
+ *                   a sliding window, one joint softmax
+ *   hca_attend      the dense (heavily compressed) variant: every visible entry
+ *
+ * Sources (page title, section):
+ *   - "DeepSeek V4とOpenCode" (hazakura.dev), "衝撃1：CSA + HCA": 4 tokens per
+ *     CSA entry, FP4 Lightning Indexer picks the top-k, 128-token sliding
+ *     window; HCA folds 128 tokens per entry and attends densely.
+ *   - jiwasawa.github.io DeepSeek-V4 article, "Compressed Sparse Attention
+ *     (CSA)" / "Heavily Compressed Attention (HCA)": sequence length becomes
+ *     1/m, indexer scores + top-k selector (DSA), shared key-value MQA over
+ *     the selected entries; HCA has m' >> m and no selection; a sliding-window
+ *     branch over recent uncompressed tokens runs alongside.
+ *   - "DeepSeek V4 Flash：知っておくべき284Bパラメータのオープンソースモデル"
+ *     (studioglobal.ai), "アテンションのブレイクスルー：CSAとHCA": softmax-
+ *     gated pooling, top 512 compressed blocks per query, HCA 128:1, window of
+ *     the latest 128 tokens.
+ *   - "DeepSeek V4 1M context window agent efficient inference"
+ *     (ai-papers.net), "ハイブリッドアテンションの仕組み": KV entries in FP8,
+ *     indexer in FP4.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   - All pointers are DEVICE pointers (cudaMalloc / torch CUDA tensors) unless
+ *     stated otherwise.  Every buffer is owned by the caller; the library never
+ *     allocates, frees or retains a pointer after the call returns.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default
+ *     stream); the library never synchronises except in csa_sync_status().
+ *   - Buffers must be 16-byte aligned and densely packed in the layouts given
+ *     (row-major, last index fastest).
+ *   - Return value: CSA_OK (0) or a negative CSA_ERR_* code.  On error nothing
+ *     was launched and csa_last_error() returns a message (thread-local).
+ *   - Formats: E4M3 = OCP FP8 E4M3 ("FN": no infinities; 0x7F/0xFF are NaN and
+ *     never written).  E2M1 = OCP MX FP4, two codes per byte, the even element
+ *     in the low nibble.  bf16 values are passed as their uint16 bit patterns.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *csa_stream_t;
+
+enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID = -1,     /* bad shape, pointer, alignment or argument     */
+  CSA_ERR_UNSUPPORTED = -2, /* valid but outside the compiled shape set      */
+  CSA_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed          */
+  CSA_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up            */
+  CSA_ERR_WORKSPACE = -5    /* workspace missing or smaller than required    */
+};
+
+/*
+ * Shapes of one attention / indexer call.
+ *   B          sequences in the batch
+ *   Tq         query rows per sequence
+ *   H          attention query heads (shared K = V, multi-query)
+ *   D          width of a KV entry; one of 64, 128, 256, 512
+ *   HI, dI     indexer heads (1..8) and indexer width (32 or 64)
+ *   K          top-k (1..2048)
+ *   W          sliding-window length in tokens (1..win_cap)
+ *   m          tokens per compressed entry (CSA: 4, HCA: 128; any m >= 1)
+ *   n_entries  valid compressed entries per sequence (cache fill level)
+ *   entry_cap  entry stride per sequence of the cache buffers (>= n_entries)
+ *   win_cap    window-ring capacity; token p sits in slot p % win_cap
+ *   softmax_scale  multiplies q . v before the softmax (1.0: folded into q)
+ */
+typedef struct csa_dims {
+  int32_t B, Tq, H, D, HI, dI, K, W, m;
+  int32_t n_entries;
+  int64_t entry_cap;
+  int32_t win_cap;
+  float softmax_scale;
+} csa_dims;
+
+/*
+ * csa_compress -- softmax-gated pooling into FP8 entries.
+ * (studioglobal.ai "アテンションのブレイクスルー：CSAとHCA": softmax-gated
+ *  pooling; hazakura.dev "衝撃1": m = 4 and m' = 128; ai-papers.net
+ *  "ハイブリッドアテンションの仕組み": FP8 KV.)
+ *
+ * For every sequence b and every FULL block i (i < T / m; a partial tail is
+ * not an entry) and channel c:
+ *     C[c]  = sum_j softmax_j(z[b, i*m + j, c]) * x[b, i*m + j, c]   (fp32)
+ *     s     = max_c |C[c]| / 448   (s = 1 if that is 0)
+ *     code  = E4M3(C[c] / s), round-to-nearest-even, saturating at +-448
+ * With m = 1 this stores single tokens (the sliding-window cache).
+ *
+ *   x, z       fp32 [B, *, D], token t of sequence b at x + b*x_batch_stride + t*D;
+ *              the first T tokens are read.
+ *   codes      u8   entry slot e of sequence b at codes + (b*dst_batch_stride + e)*D
+ *   scales     fp32 scale of that entry at scales[b*dst_batch_stride + e]
+ *   dst_first  slot of block 0; block i goes to slot dst_first + i, taken modulo
+ *              ring_cap when ring_cap > 0 (ring buffer), else used as is.
+ *   pooled     optional fp32 [B, T/m, D] copy of C before quantisation (NULL = none)
+ * Requires D % 4 == 0, 4 <= D <= 1024, m >= 1, T >= 0; T < m is a no-op.
+ */
+int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D, int32_t m,
+                 int64_t x_batch_stride, uint8_t *codes, float *scales, int64_t dst_first,
+                 int64_t dst_batch_stride, int32_t ring_cap, float *pooled,
+                 csa_stream_t stream);
+
+/*
+ * csa_index_topk -- Lightning-Indexer scores and top-k.
+ * (jiwasawa "Compressed Sparse Attention (CSA)": indexer scores per query and
+ *  a top-k selector; hazakura.dev "衝撃1": FP4 indexer; studioglobal.ai
+ *  "アテンションのブレイクスルー": top 512 blocks per query.)
+ *
+ * For query row (b, i) at position t = q_pos[b, i], entry s is visible iff
+ * s < n_vis = min(floor((t + 1) / m), n_entries).  Its score is
+ *     score = sum_h w[b,i,h] * max(0, sum_j qI[b,i,h,j] * kI[b,s,j])
+ * computed exactly (E2M1 products are multiples of 1/4; w must be a multiple
+ * of 1/16 in [0, 1], so 64*score is an integer below 2^24).  The row's output
+ * lists the min(K, n_vis) best entries in rank order -- score descending, ties
+ * to the lower index -- followed by -1 padding.
+ *
+ *   qI         u8   [B, Tq, HI, dI/2]   packed E2M1
+ *   w          fp32 [B, Tq, HI]
+ *   kI         u8   [B, entry_cap, dI/2] packed E2M1
+ *   q_pos      int32 [B, Tq]             (>= 0)
+ *   idx_out    int32 [B, Tq, K]
+ *   score_out  fp32 [B, Tq, K] scores of the listed entries (0 for padding), or NULL
+ *   workspace  device scratch of at least csa_index_topk_workspace(d) bytes
+ * Uses d->B, Tq, HI, dI, K, m, n_entries, entry_cap.
+ */
+size_t csa_index_topk_workspace(const csa_dims *d);
+int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+                   const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
+                   size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * csa_attend -- sparse shared-KV MQA over selected entries + window.
+ * (jiwasawa "Compressed Sparse Attention (CSA)": shared key-value MQA over
+ *  the selected entries; "Heavily Compressed Attention (HCA)": the sliding
+ *  window branch; studioglobal.ai: the window is the latest 128 tokens.)
+ *
+ * For query row (b, i) at position t = q_pos[b, i] the key/value set is
+ *     U = { entry idx[b,i,j] : idx >= 0 }  +  { window token p : max(0,t-W+1) <= p <= t }
+ * (no de-duplication), each row dequantised as code * scale, K = V.  For every
+ * head h: S_u = softmax_scale * q[b,i,h,:] . U_u,  out = sum_u softmax(S)_u U_u,
+ * lse = max S + ln(sum exp(S - max S)).
+ *
+ *   q          bf16 [B, Tq, H, D]
+ *   codes      u8   [B, entry_cap, D], scales fp32 [B, entry_cap]   (csa_compress output)
+ *   idx        int32 [B, Tq, K]  (entries must be < n_entries; -1 = unused)
+ *   win_codes  u8   [B, win_cap, D], win_scales fp32 [B, win_cap]   (m = 1 entries)
+ *   q_pos      int32 [B, Tq]
+ *   out        bf16 [B, Tq, H, D];  lse fp32 [B, Tq, H] or NULL
+ *   workspace  device scratch of at least csa_attend_workspace(d) bytes
+ * Requires W <= win_cap (every window token still resident in the ring).
+ */
+size_t csa_attend_workspace(const csa_dims *d);
+int csa_attend(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
+               const uint8_t *win_codes, const float *win_scales, const int32_t *q_pos,
+               const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+               size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * hca_attend -- dense attention over every visible entry + window.
+ * (jiwasawa "Heavily Compressed Attention (HCA)": no sparse selection, dense
+ *  attention over the compressed sequence; hazakura.dev "衝撃1": m' = 128.)
+ * As csa_attend with the selection replaced by all entries s < n_vis(t) =
+ * min(floor((t+1)/m), n_entries).  Same buffers minus idx.
+ */
+size_t hca_attend_workspace(const csa_dims *d);
+int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
+               const uint8_t *win_codes, const float *win_scales, const int32_t *q_pos,
+               const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+               size_t workspace_bytes, csa_stream_t stream);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char *csa_last_error(void);
+
+/*
+ * Waits for `stream`, then reads and clears the library's device status word,
+ * which kernels set when a bounded device-side wait gives up.  Returns CSA_OK,
+ * CSA_ERR_TIMEOUT, or CSA_ERR_CUDA if the stream itself reported an error.
+ */
+int csa_sync_status(csa_stream_t stream);
+
+/* Library ABI version (major * 100 + minor). */
+int csa_version(void);
+
+/* Number of GPU kernels this library has launched in this process (all
+ * devices, all threads) -- for accounting in benchmarks and tests. */
+uint64_t csa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H */

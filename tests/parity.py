@@ -1,0 +1,96 @@
+"""Comparison rules shared by the GPU parity tests.
+
+Tolerances (derived from the arithmetic; the numeric bars are the library's
+contract):
+* indexer scores and top-k indices: bit-exact (the scores are exact integers
+  in units of 1/64 on both sides).
+* pooled fp32 value of channel c: |gpu - ref| <= 1e-5 * A_c, where
+  A_c = sum_i p_i |x_i| is the natural scale of a weighted sum (the fp32
+  bound for m <= 128 terms is about (m + 3) * 2^-24 * A_c < 1e-5 * A_c).
+* E4M3 codes: equal, except a flip to the NEIGHBOURING code where the
+  oracle's fp32 ratio r = C/s lies within delta of the midpoint between the
+  two codes; delta is what the pooled tolerance allows r to move:
+  delta = 1e-5 * A_c / s + |r| * 1e-5 * A_amax / amax + 2^-22 |r|.
+* scales: |gpu - ref| <= 1e-5 * A_amax / 448 + 2^-23 * ref.
+* attention output (bf16): per query row and head, max_d |gpu - ref| <=
+  1e-2 * max_d |ref|.
+* log-sum-exp: |gpu - ref| <= 1e-4 (logits are exact products of bf16 and
+  E4M3 values accumulated in fp32; exp2/log2 add a few ulp).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from oracle import csa as ocsa
+from oracle.formats import e4m3_decode
+
+POOL_RTOL = 1e-5
+OUT_RTOL = 1e-2
+LSE_ATOL = 1e-4
+
+
+def pooled_and_scale(x, z, m):
+    """Oracle pooled values (fp64) and A = pool(|x|) for full blocks of x, z [B, T, D]."""
+    ref = ocsa.compress(x, z, m)
+    A = ocsa.compress(np.abs(np.asarray(x, dtype=np.float64)), z, m)
+    return ref, A
+
+
+def check_pooled(gpu, ref, A):
+    err = np.abs(np.asarray(gpu, dtype=np.float64) - ref)
+    bad = err > POOL_RTOL * A + 1e-30
+    assert not bad.any(), f"pooled mismatch at {np.argwhere(bad)[:5].tolist()}: max err/A {(err / A).max():.3g}"
+
+
+def check_codes(gpu_codes, gpu_scales, ref_pooled, A):
+    """Compare GPU codes/scales with the oracle's quantisation of its own pooled values."""
+    ref_codes, ref_s = ocsa.quantize_entries(ref_pooled)
+    r = ocsa.quantize_ratio(ref_pooled)
+    gpu_codes = np.asarray(gpu_codes)
+    gpu_scales = np.asarray(gpu_scales, dtype=np.float64)
+    amax = np.abs(ref_pooled.astype(np.float32)).max(axis=-1).astype(np.float64)
+    amax_ch = np.abs(ref_pooled.astype(np.float32)).argmax(axis=-1)
+    A_amax = np.take_along_axis(A, amax_ch[..., None], axis=-1)[..., 0]
+    s = ref_s.astype(np.float64)
+    # scales
+    tol_s = POOL_RTOL * A_amax / 448.0 + 2.0 ** -23 * s
+    bad = np.abs(gpu_scales - s) > tol_s
+    assert not bad.any(), f"scale mismatch at {np.argwhere(bad)[:5].tolist()}"
+    # codes
+    diff = gpu_codes != ref_codes
+    n_flip = int(diff.sum())
+    if n_flip:
+        vg = e4m3_decode(gpu_codes[diff])
+        vr = e4m3_decode(ref_codes[diff])
+        rr = r[diff]
+        finite = e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+        lo = np.minimum(np.abs(vg), np.abs(vr))
+        hi = np.maximum(np.abs(vg), np.abs(vr))
+        # neighbours: no finite magnitude strictly between them, same sign unless one is zero
+        between = ((finite[None, :] > lo[:, None]) & (finite[None, :] < hi[:, None])).any(axis=1)
+        same_sign = (np.sign(vg) == np.sign(vr)) | (vg == 0) | (vr == 0)
+        mid = (lo + hi) / 2.0
+        Ad = np.broadcast_to(A, r.shape)[diff]
+        sd = np.broadcast_to(s[..., None], r.shape)[diff]
+        eps_s = np.broadcast_to((POOL_RTOL * A_amax / amax.clip(1e-300))[..., None], r.shape)[diff]
+        delta = POOL_RTOL * Ad / sd + np.abs(rr) * eps_s + 2.0 ** -22 * np.abs(rr)
+        ok = ~between & same_sign & (np.abs(np.abs(rr) - mid) <= delta)
+        assert ok.all(), (f"{int((~ok).sum())} code mismatches are not near-midpoint flips, e.g. "
+                          f"gpu={gpu_codes[diff][~ok][:5]} ref={ref_codes[diff][~ok][:5]} r={rr[~ok][:5]}")
+    return n_flip
+
+
+def check_attention(gpu_out_bf16, gpu_lse, ref_out, ref_lse):
+    import torch
+    g = gpu_out_bf16.float().cpu().numpy().astype(np.float64) if isinstance(gpu_out_bf16, torch.Tensor) \
+        else np.asarray(gpu_out_bf16, dtype=np.float64)
+    err = np.abs(g - ref_out).max(axis=-1)
+    scale = np.abs(ref_out).max(axis=-1)
+    bad = err > OUT_RTOL * scale
+    assert not bad.any(), (f"attention mismatch at {np.argwhere(bad)[:5].tolist()}: "
+                           f"worst err/max|ref| = {(err / scale).max():.3g}")
+    if gpu_lse is not None:
+        gl = gpu_lse.cpu().numpy().astype(np.float64) if hasattr(gpu_lse, "cpu") else np.asarray(gpu_lse)
+        lerr = np.abs(gl - ref_lse)
+        assert lerr.max() <= LSE_ATOL, f"lse mismatch: max err {lerr.max():.3g}"
+    return float((err / scale).max())

@@ -1,0 +1,147 @@
+"""GPU parity of csa_attend / hca_attend against the oracle's fp64 attention,
+through the C ABI.  The compressed cache and the window ring are random E4M3
+bytes from the seeded generator (the same bytes go to both sides)."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_attention_16_b200 as csa
+import synth
+from compressed_sparse_attention_16_b200 import Dims
+from oracle import csa as ocsa
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def _random_selection(rng, q_pos, m, n_entries, K, pad_anywhere=False):
+    B, Tq = q_pos.shape
+    idx = np.full((B, Tq, K), -1, dtype=np.int32)
+    for b in range(B):
+        for i in range(Tq):
+            nv = int(ocsa.n_visible(q_pos[b, i], m, n_entries))
+            k = min(K, nv)
+            if k:
+                pick = rng.choice(nv, k, replace=False)
+                if pad_anywhere:
+                    slots = np.sort(rng.choice(K, k, replace=False))
+                    idx[b, i, slots] = pick
+                else:
+                    idx[b, i, :k] = pick
+    return idx
+
+
+def _setup(B, Tq, H, D, N, win_cap, q_pos, seed, q_scale):
+    codes, scales = synth.e4m3_cache(B, N, D, seed)
+    wcodes, wscales = synth.e4m3_cache(B, win_cap, D, seed, tag="win")
+    q = synth.queries(B, Tq, H, D, q_scale, seed)
+    ent = ocsa.dequantize(codes.numpy(), scales.numpy())
+    wv = ocsa.dequantize(wcodes.numpy(), wscales.numpy())
+    return codes, scales, wcodes, wscales, q, ent, wv
+
+
+def _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d):
+    B, Tq, H, D = q.shape
+    out = torch.empty((B, Tq, H, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Tq, H), device="cuda")
+    dense = idx is None
+    nb = csa.attend_workspace(d, dense)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+    args = (q.cuda(), codes.cuda(), scales.cuda())
+    tail = (wcodes.cuda(), wscales.cuda(), torch.from_numpy(q_pos).cuda(), d, out, lse)
+    if dense:
+        csa.hca_attend(*args, *tail, workspace=ws)
+    else:
+        csa.attend(*args, torch.from_numpy(idx).cuda(), *tail, workspace=ws)
+    csa.sync_status()
+    return out, lse
+
+
+CASES = [
+    # B, Tq, H, D, m, N, K, W, win_cap, q_scale
+    (2, 7, 4, 64, 4, 128, 16, 32, 512, 1 / 8),
+    (2, 5, 128, 512, 4, 3000, 512, 128, 128, 512 ** -0.5),
+    (1, 9, 64, 512, 4, 2100, 512, 128, 8400, 512 ** -0.5),
+    (3, 4, 16, 256, 4, 700, 100, 50, 64, 0.1),
+    (1, 6, 8, 128, 2, 400, 33, 7, 7, 0.2),
+]
+
+
+@pytest.mark.parametrize("B,Tq,H,D,m,N,K,W,win_cap,qs", CASES)
+def test_csa_attend_parity(B, Tq, H, D, m, N, K, W, win_cap, qs):
+    rng = np.random.default_rng(B * 100 + H + D)
+    tmax = min(m * N + m - 1, win_cap * 50)
+    q_pos = rng.integers(0, tmax, (B, Tq)).astype(np.int32)
+    q_pos[0, 0] = 0
+    q_pos[-1, -1] = m * N - 1
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, Tq, H, D, N, win_cap, q_pos, 7, qs)
+    idx = _random_selection(rng, q_pos, m, N, K, pad_anywhere=(K == 100))
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=win_cap)
+    out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % win_cap], q_pos, W)
+    parity.check_attention(out, lse, ro, rl)
+
+
+@pytest.mark.parametrize("B,Tq,H,D,m,N,W", [(2, 5, 128, 512, 128, 300, 128), (1, 4, 4, 64, 4, 200, 32),
+                                             (2, 3, 64, 512, 4, 1500, 128)])
+def test_hca_attend_parity(B, Tq, H, D, m, N, W):
+    rng = np.random.default_rng(N)
+    q_pos = rng.integers(0, m * N + 3 * m, (B, Tq)).astype(np.int32)
+    q_pos[0, 0] = m - 2          # before the first entry completes: window only
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, Tq, H, D, N, W, q_pos, 8, 512 ** -0.5)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=1, W=W, m=m, n_entries=N, win_cap=W)
+    out, lse = _run_gpu(q, codes, scales, None, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.hca_attend(_bits(q), ent, lambda b, p: wv[b, p % W], q_pos, m, W)
+    parity.check_attention(out, lse, ro, rl)
+
+
+def test_softmax_scale_is_applied():
+    B, Tq, H, D, m, N, K, W = 1, 3, 8, 64, 4, 50, 8, 16
+    q_pos = np.array([[199, 100, 40]], dtype=np.int32)
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, Tq, H, D, N, W, q_pos, 9, 1.0)
+    idx = _random_selection(np.random.default_rng(3), q_pos, m, N, K)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=W, softmax_scale=0.125)
+    out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % W], q_pos, W, scale=0.125)
+    parity.check_attention(out, lse, ro, rl)
+
+
+def test_out_of_range_index_is_reported():
+    B, Tq, H, D, m, N, K, W = 1, 1, 4, 64, 4, 20, 4, 8
+    q_pos = np.array([[79]], dtype=np.int32)
+    codes, scales, wcodes, wscales, q, _, _ = _setup(B, Tq, H, D, N, W, q_pos, 10, 0.1)
+    idx = np.array([[[1, 2, 20, -1]]], dtype=np.int32)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=W)
+    with pytest.raises(csa.CsaError) as e:
+        _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    assert e.value.code == csa.CSA_ERR_INVALID
+
+
+def test_csa_decode_64k_full_size():
+    """Attention step of the 64K-context decode workload: 16 sequences, 128
+    heads, D = 512, K = 512 selected of 16,384 entries plus a 128-token window."""
+    B, H, D, m, N, K, W = 16, 128, 512, 4, 16384, 512, 128
+    rng = np.random.default_rng(12)
+    q_pos = np.full((B, 1), m * N - 1, dtype=np.int32)
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, 1, H, D, N, W, q_pos, 12, 512 ** -0.5)
+    idx = _random_selection(rng, q_pos, m, N, K)
+    d = Dims(B=B, Tq=1, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=W)
+    out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % W], q_pos, W)
+    parity.check_attention(out, lse, ro, rl)
+
+
+def test_hca_decode_1m_full_size():
+    """Attention step of the 1M-context HCA workload: 16 sequences x (8,192
+    entries + 128 window tokens) x 128 heads x 512."""
+    B, H, D, m, N, W = 16, 128, 512, 128, 8192, 128
+    q_pos = np.full((B, 1), m * N - 1, dtype=np.int32)
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, 1, H, D, N, W, q_pos, 13, 512 ** -0.5)
+    d = Dims(B=B, Tq=1, H=H, D=D, K=1, W=W, m=m, n_entries=N, win_cap=W)
+    out, lse = _run_gpu(q, codes, scales, None, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.hca_attend(_bits(q), ent, lambda b, p: wv[b, p % W], q_pos, m, W)
+    parity.check_attention(out, lse, ro, rl)
