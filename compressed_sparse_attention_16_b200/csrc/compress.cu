@@ -59,13 +59,17 @@ compress_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_
   const int g = threadIdx.x / L;
   const int lane = threadIdx.x - g * L;
   const int64_t e = (int64_t)blockIdx.x * groups + g;
-  const bool active = (g < groups) && (e < n_total);
-
-  float C[4] = {0.f, 0.f, 0.f, 0.f};
   int64_t b = 0, i = 0;
-  if (active) {
+  if (g < groups && e < n_total) {
     b = e / n_per_seq;
     i = e - b * n_per_seq;
+  }
+  // With a ring of ring_cap slots only the call's last ring_cap blocks survive;
+  // earlier blocks would share their slots, so they are not written at all.
+  const bool active = (g < groups) && (e < n_total) && !(ring_cap > 0 && i + ring_cap < n_per_seq);
+
+  float C[4] = {0.f, 0.f, 0.f, 0.f};
+  if (active) {
     const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + lane;
     const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + lane;
     OnlineSoftmax4 sm;

@@ -105,7 +105,9 @@ typedef struct csa_dims {
  *   codes      u8   entry slot e of sequence b at codes + (b*dst_batch_stride + e)*D
  *   scales     fp32 scale of that entry at scales[b*dst_batch_stride + e]
  *   dst_first  slot of block 0; block i goes to slot dst_first + i, taken modulo
- *              ring_cap when ring_cap > 0 (ring buffer), else used as is.
+ *              ring_cap when ring_cap > 0 (ring buffer), else used as is.  With
+ *              a ring, only the call's last ring_cap blocks are pooled and
+ *              stored (earlier ones would be overwritten by them).
  *   pooled     optional fp32 [B, T/m, D] copy of C before quantisation (NULL = none)
  * Requires D % 4 == 0, 4 <= D <= 1024, m >= 1, T >= 0; T < m is a no-op.
  */

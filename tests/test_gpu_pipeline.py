@@ -22,6 +22,8 @@ def _bits(t):
 def _entry_values(x, z, b, entries, m):
     """Oracle entries (dequantised) for the given entry ids of sequence b;
     x, z may live on the GPU -- only the needed tokens are copied."""
+    if len(entries) == 0:
+        return np.zeros((0, x.shape[-1]))
     e = torch.as_tensor(np.asarray(entries, dtype=np.int64), device=x.device)
     tok = (e[:, None] * m + torch.arange(m, device=x.device)[None]).reshape(-1)
     xs = x[b, tok].reshape(len(entries), m, -1).cpu().numpy()
