@@ -128,3 +128,11 @@ def test_prefill_full_size_sampled_rows():
                           torch.from_numpy(rows[None].astype(np.int32)), m, K, N)
     assert np.array_equal(idx[:, r].cpu().numpy(), ri)
     assert np.array_equal(sc[:, r].cpu().numpy().astype(np.float64), rs)
+
+
+def test_negative_position_is_reported():
+    B, Tq, N = 1, 2, 64
+    inp = synth.indexer_inputs(B, Tq, N, 4, 64, seed=8)
+    with pytest.raises(csa.CsaError) as e:
+        _gpu_topk(inp.qI, inp.w, inp.kI, torch.tensor([[-5, 10]], dtype=torch.int32), 4, 8, N)
+    assert e.value.code == csa.CSA_ERR_INVALID
