@@ -29,6 +29,7 @@ SYMBOLS = (
     "csa_compress",
     "csa_index_topk_workspace",
     "csa_index_topk",
+    "csa_index_topk_noalloc",
     "csa_attend_workspace",
     "csa_attend",
     "hca_attend_workspace",
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.csa_index_topk_workspace.restype = _SZ
     L.csa_index_topk.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
     L.csa_index_topk.restype = ctypes.c_int
+    L.csa_index_topk_noalloc.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P]
+    L.csa_index_topk_noalloc.restype = ctypes.c_int
     for name in ("csa_attend_workspace", "hca_attend_workspace"):
         getattr(L, name).argtypes = [ctypes.POINTER(Dims)]
         getattr(L, name).restype = _SZ
@@ -184,6 +187,18 @@ def index_topk(qI, w, kI, q_pos, dims: Dims, idx_out, score_out=None, workspace=
                                 _ptr(kI, torch.uint8, "kI", dev), _ptr(q_pos, torch.int32, "q_pos", dev),
                                 ctypes.byref(dims), _ptr(idx_out, torch.int32, "idx_out", dev),
                                 _ptr(score_out, torch.float32, "score_out", dev), wp, wn, _stream(stream)))
+
+
+def index_topk_noalloc(qI, w, kI, q_pos, dims: Dims, idx_out, score_out=None, stream=None):
+    """csa_index_topk_noalloc: as index_topk, but the library's own fixed 8 MiB
+    device scratch replaces the workspace (for callers that cannot allocate).
+    Calls that overlap on the GPU share that scratch and must be serialised."""
+    dev = qI.device
+    _check(lib().csa_index_topk_noalloc(_ptr(qI, torch.uint8, "qI"), _ptr(w, torch.float32, "w", dev),
+                                        _ptr(kI, torch.uint8, "kI", dev),
+                                        _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
+                                        _ptr(idx_out, torch.int32, "idx_out", dev),
+                                        _ptr(score_out, torch.float32, "score_out", dev), _stream(stream)))
 
 
 def attend(q, codes, scales, idx, win_codes, win_scales, q_pos, dims: Dims, out, lse=None,

@@ -145,6 +145,31 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
                    size_t workspace_bytes, csa_stream_t stream);
 
 /*
+ * csa_index_topk_noalloc -- csa_index_topk without a caller-provided workspace.
+ * (The pages have no counterpart: this is a deployment convenience.)
+ *
+ * For callers that cannot allocate device memory -- code inside allocator
+ * hooks, runtimes that plan every byte at load time and forbid cudaMalloc
+ * afterwards, plug-ins that only receive their inputs' and outputs' buffers.
+ * Same arguments, results and errors as csa_index_topk, minus the workspace:
+ * the scratch is an 8 MiB array inside the library's device image, held by
+ * every GPU that loads the library until the process exits.  Shapes whose
+ * workspace (csa_index_topk_workspace) exceeds 8 MiB -- e.g. more than 2M
+ * (query row x entry) pairs -- are rejected with CSA_ERR_UNSUPPORTED before
+ * any launch.  The library allocates nothing and calls no allocating routine.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - All calls share the one array: calls whose kernels overlap on the GPU
+ *     (different streams, or different host threads) race and corrupt each
+ *     other's results; serialise them.  Stale contents from an earlier call
+ *     are harmless (every score is written before it is read).
+ */
+int csa_index_topk_noalloc(const uint8_t *qI, const float *w, const uint8_t *kI,
+                           const int32_t *q_pos, const csa_dims *d, int32_t *idx_out,
+                           float *score_out, csa_stream_t stream);
+
+/*
  * csa_attend -- sparse shared-KV MQA over selected entries + window.
  * (jiwasawa "Compressed Sparse Attention (CSA)": shared key-value MQA over
  *  the selected entries; "Heavily Compressed Attention (HCA)": the sliding
