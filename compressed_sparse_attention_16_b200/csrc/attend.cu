@@ -224,13 +224,23 @@ int launch_generic(const __nv_bfloat16 *q, const uint8_t *codes, const float *sc
 
 }  // namespace
 
+bool attend_tc_supported(const csa_dims *d);
+size_t attend_tc_workspace(const csa_dims *d, bool dense);
+int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
+                     const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
+                     const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+                     cudaStream_t stream);
+
+// 128 heads x 512-wide entries run on the tensor cores; other shapes use the
+// generic CUDA-core kernel above.
 int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
                   const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
                   const csa_dims *d, uint16_t *out, float *lse, void *workspace, size_t ws_bytes,
                   cudaStream_t stream) {
-  (void)workspace;
   (void)ws_bytes;
   if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
+  if (attend_tc_supported(d))
+    return launch_attend_tc(q, codes, scales, idx, wcodes, wscales, q_pos, d, out, lse, workspace, stream);
   const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
   auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
   switch (d->D) {
@@ -245,10 +255,9 @@ int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, 
 }  // namespace csa
 
 namespace csa {
-// The generic kernel keeps its whole softmax state on chip: no scratch.
+// The generic kernel keeps its whole softmax state on chip; the tensor-core
+// kernel needs scratch for split partial outputs when a row is split.
 size_t attend_workspace(const csa_dims *d, bool dense) {
-  (void)d;
-  (void)dense;
-  return 0;
+  return attend_tc_supported(d) ? attend_tc_workspace(d, dense) : 0;
 }
 }  // namespace csa
