@@ -153,24 +153,26 @@ class ClockSampler:
 
 
 class Runner:
-    """Holds one workload's device state and runs steps of it."""
+    """One workload's device state.  `calls(i)` lists the library calls of step i
+    as (name, launch) pairs; a step is replayed as one CUDA graph."""
 
     def __init__(self, wl, seed, device):
         import torch
 
         import synth
-        from compressed_sparse_attention_16_b200 import pipeline
+        from compressed_sparse_attention_16_b200 import Dims, pipeline
 
         self.torch = torch
         self.wl = wl
         self.dev = device
         torch.cuda.set_device(device)
-        self.calls = {}
-        if wl.kind in ("decode", "decode_incremental", "hca_decode"):
-            self.n_new = 4 if wl.kind != "hca_decode" else wl.m
-            steps_cap = max(wl.steps, 1) + 1024 if wl.kind == "decode_incremental" else 1
+        self.graphs = {}
+        self.decode = wl.kind in ("decode", "decode_incremental", "hca_decode")
+        if self.decode:
+            self.n_new = wl.m if wl.kind == "hca_decode" else 4
+            self.n_steps = max(wl.steps, 1) + 256 if wl.kind == "decode_incremental" else 1
             self.T0 = wl.T if wl.kind == "decode_incremental" else wl.T - self.n_new
-            Ttot = self.T0 + self.n_new * steps_cap
+            Ttot = self.T0 + self.n_new * self.n_steps
             self.x, self.z = synth.tokens(wl.B, Ttot, wl.D, seed, device=device)
             dense = wl.kind == "hca_decode"
             cap = Ttot // wl.m
@@ -181,9 +183,21 @@ class Runner:
                 self.state.kI.copy_(self.ind.kI)
             self.q = synth.queries(wl.B, 1, wl.H, wl.D, wl.q_scale, seed, device=device)
             self.state.prefill_context(self.x, self.z, self.T0)
-            self.step_i = 0
+            # per-step query positions (graph-static)
+            pos = self.T0 + self.n_new * (torch.arange(self.n_steps, device=device) + 1) - 1
+            self.q_pos_all = pos.to(torch.int32)[:, None, None].repeat(1, wl.B, 1).contiguous()
             self.units_per_step = wl.B
             self.unit = "tokens/s"
+            self.Dims = Dims
+            # workspaces sized for the largest step, allocated before any capture
+            import compressed_sparse_attention_16_b200 as csa
+            for j in (0, self.n_steps - 1):
+                d = self._dims(j)
+                if wl.kind == "hca_decode":
+                    self._ws(csa.attend_workspace(d, True), "_ws_hca")
+                else:
+                    self._ws(csa.index_topk_workspace(d), "_ws_index")
+                    self._ws(csa.attend_workspace(d), "_ws_attend")
         else:
             self.x, self.z = synth.tokens(wl.B, wl.T, wl.D, seed, device=device)
             self.q = synth.queries(wl.B, wl.T, wl.H, wl.D, wl.q_scale, seed, device=device)
@@ -213,82 +227,99 @@ class Runner:
         nb = csa.attend_workspace(self.dims)
         self.ws_a = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
 
-    # -- one step, each library call bracketed by events when `ev` is given ----
-    def _call(self, name, ev, fn):
-        if ev is None:
-            fn()
-            return
-        e0 = self.torch.cuda.Event(enable_timing=True)
-        e1 = self.torch.cuda.Event(enable_timing=True)
-        e0.record()
-        fn()
-        e1.record()
-        ev.append((name, e0, e1))
+    def _ws(self, nbytes, key):
+        cur = getattr(self, key, None)
+        if nbytes and (cur is None or cur.numel() < nbytes):
+            if self.torch.cuda.is_current_stream_capturing():
+                raise RuntimeError("workspace growth during graph capture")
+            cur = self.torch.empty(int(nbytes * 1.25) + 4096, dtype=self.torch.uint8, device=self.dev)
+            setattr(self, key, cur)
+        return cur if nbytes else None
 
-    def _decode_t0(self):
-        if self.wl.kind == "decode_incremental":
-            return self.T0 + self.n_new * self.step_i
-        return self.T0            # decode / hca_decode: the same last block every step
+    def _dims(self, j):
+        wl, st = self.wl, self.state
+        t0 = self.T0 + self.n_new * j
+        return self.Dims(B=wl.B, Tq=1, H=wl.H, D=wl.D, HI=st.HI, dI=st.dI, K=st.K, W=wl.W, m=wl.m,
+                         n_entries=(t0 + self.n_new) // wl.m, entry_cap=st.entry_cap, win_cap=st.win_cap)
 
-    def step(self, ev=None, inputs=None):
-        """One step on the current stream; q_pos was set by prepare_step()."""
+    def step_index(self, i):
+        return i % self.n_steps if self.wl.kind == "decode_incremental" else 0
+
+    def calls(self, i, inputs=None):
+        """(name, launch) pairs of step i.  `inputs` (optional) supplies contiguous
+        device buffers x, z [B, n_new, D], q, qI, w instead of the resident ones."""
         import compressed_sparse_attention_16_b200 as csa
         wl = self.wl
-        if wl.kind in ("decode", "decode_incremental", "hca_decode"):
-            st = self.state
-            t0 = self._decode_t0()
-            st.n_tokens = t0
-            xs = (self.x[:, t0:t0 + self.n_new] if inputs is None else inputs["x"]).contiguous()
-            zs = (self.z[:, t0:t0 + self.n_new] if inputs is None else inputs["z"]).contiguous()
+        if not self.decode:
+            x = self.x if inputs is None else inputs["x"]
+            z = self.z if inputs is None else inputs["z"]
             q = self.q if inputs is None else inputs["q"]
-            first = st.n_entries
-            self._call("compress_entry", ev, lambda: csa.compress(xs, zs, wl.m, st.codes, st.scales, dst_first=first))
-            self._call("compress_window", ev, lambda: csa.compress(xs, zs, 1, st.win_codes, st.win_scales,
-                                                                    dst_first=t0, ring_cap=st.win_cap))
-            st.n_tokens = t0 + self.n_new
-            if wl.kind == "decode_incremental":
-                self.step_i += 1
-            d = st.dims()
-            if wl.kind == "hca_decode":
-                self._call("hca_attend", ev, lambda: csa.hca_attend(q, st.codes, st.scales, st.win_codes,
-                                                                    st.win_scales, st.q_pos, d, st.out, st.lse,
-                                                                    workspace=self._ws(d, "attend_dense")))
-            else:
-                qI = self.ind.qI if inputs is None else inputs["qI"]
-                w = self.ind.w if inputs is None else inputs["w"]
-                self._call("index_topk", ev, lambda: csa.index_topk(qI, w, st.kI, st.q_pos, d, st.idx, st.score,
-                                                                    workspace=self._ws(d, "index")))
-                self._call("attend", ev, lambda: csa.attend(q, st.codes, st.scales, st.idx, st.win_codes,
-                                                            st.win_scales, st.q_pos, d, st.out, st.lse,
-                                                            workspace=self._ws(d, "attend")))
-            return st.out
-        x = self.x if inputs is None else inputs["x"]
-        z = self.z if inputs is None else inputs["z"]
+            return [
+                ("compress_entry", lambda: csa.compress(x, z, wl.m, self.codes, self.scales)),
+                ("compress_window", lambda: csa.compress(x, z, 1, self.wcodes, self.wscales)),
+                ("index_topk", lambda: csa.index_topk(self.ind.qI, self.ind.w, self.ind.kI, self.q_pos, self.dims,
+                                                      self.idx, self.score, workspace=self.ws_i)),
+                ("attend", lambda: csa.attend(q, self.codes, self.scales, self.idx, self.wcodes, self.wscales,
+                                              self.q_pos, self.dims, self.out, self.lse, workspace=self.ws_a)),
+            ]
+        st = self.state
+        j = self.step_index(i)
+        t0 = self.T0 + self.n_new * j
+        d = self._dims(j)
+        q_pos = self.q_pos_all[j]
+        if inputs is None:
+            src, first = (self.x, self.z), t0
+        else:
+            src, first = (inputs["x"], inputs["z"]), 0
         q = self.q if inputs is None else inputs["q"]
-        self._call("compress_entry", ev, lambda: csa.compress(x, z, wl.m, self.codes, self.scales))
-        self._call("compress_window", ev, lambda: csa.compress(x, z, 1, self.wcodes, self.wscales))
-        self._call("index_topk", ev, lambda: csa.index_topk(self.ind.qI, self.ind.w, self.ind.kI, self.q_pos,
-                                                            self.dims, self.idx, self.score, workspace=self.ws_i))
-        self._call("attend", ev, lambda: csa.attend(q, self.codes, self.scales, self.idx, self.wcodes,
-                                                    self.wscales, self.q_pos, self.dims, self.out, self.lse,
-                                                    workspace=self.ws_a))
-        return self.out
+        out = [
+            ("compress_entry", lambda: csa.compress(src[0], src[1], wl.m, st.codes, st.scales, dst_first=t0 // wl.m,
+                                                    T=self.n_new, first_token=first)),
+            ("compress_window", lambda: csa.compress(src[0], src[1], 1, st.win_codes, st.win_scales, dst_first=t0,
+                                                     ring_cap=st.win_cap, T=self.n_new, first_token=first)),
+        ]
+        if wl.kind == "hca_decode":
+            ws = self._ws(csa.attend_workspace(d, True), "_ws_hca")
+            out.append(("hca_attend", lambda: csa.hca_attend(q, st.codes, st.scales, st.win_codes, st.win_scales,
+                                                             q_pos, d, st.out, st.lse, workspace=ws)))
+        else:
+            qI = self.ind.qI if inputs is None else inputs["qI"]
+            w = self.ind.w if inputs is None else inputs["w"]
+            wsi = self._ws(csa.index_topk_workspace(d), "_ws_index")
+            wsa = self._ws(csa.attend_workspace(d), "_ws_attend")
+            out.append(("index_topk", lambda: csa.index_topk(qI, w, st.kI, q_pos, d, st.idx, st.score, workspace=wsi)))
+            out.append(("attend", lambda: csa.attend(q, st.codes, st.scales, st.idx, st.win_codes, st.win_scales,
+                                                     q_pos, d, st.out, st.lse, workspace=wsa)))
+        return out
 
-    def _ws(self, d, kind):
+    def output(self):
+        return self.state.out if self.decode else self.out
+
+    def run(self, i, inputs=None):
+        for _, fn in self.calls(i, inputs):
+            fn()
+
+    def graph(self, i, inputs=None, key=None):
+        """CUDA graph of step i (captured once)."""
         import compressed_sparse_attention_16_b200 as csa
-        nb = csa.index_topk_workspace(d) if kind == "index" else csa.attend_workspace(d, kind == "attend_dense")
-        key = "_ws_" + kind
-        cur = getattr(self, key, None)
-        if nb and (cur is None or cur.numel() < nb):
-            cur = self.torch.empty(int(nb * 1.05) + 256, dtype=self.torch.uint8, device=self.dev)
-            setattr(self, key, cur)
-        return cur if nb else None
-
-    def prepare_step(self):
-        """Set the decode query position for the next step (a device write issued
-        before the step's events)."""
-        if self.wl.kind in ("decode", "decode_incremental", "hca_decode"):
-            self.state.q_pos.fill_(self._decode_t0() + self.n_new - 1)
+        torch = self.torch
+        key = (self.step_index(i), key)
+        g = self.graphs.get(key)
+        if g is None:
+            calls = self.calls(i, inputs)
+            if not getattr(self, "_warmed", False):
+                for _, fn in calls:             # first launches set kernel attributes
+                    fn()
+                torch.cuda.synchronize()
+                self._warmed = True
+            g = torch.cuda.CUDAGraph()
+            n0 = csa.launch_count()
+            with torch.cuda.graph(g):
+                for _, fn in calls:
+                    fn()
+            g.kernels = csa.launch_count() - n0
+            self.graphs[key] = g
+        return g
 
 
 def gpu_arm(args, wl):
@@ -307,42 +338,50 @@ def gpu_arm(args, wl):
     peaks, peaks_src = load_peaks()
     r = Runner(wl, seed=rank, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    use_graph = r.decode and not args.no_graph
 
     def barrier():
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        r.prepare_step()
-        r.step()
+    # warm-up (also captures the graphs of the steps to be timed)
+    for i in range(args.warmup):
+        if use_graph:
+            r.graph(i).replay()
+        else:
+            r.run(i)
+    if use_graph:
+        for i in range(args.warmup, args.warmup + args.steps):
+            r.graph(i)
     barrier()
+
     clocks = ClockSampler(local)
     clocks.start()
-    evs = []
     step_events = []
-    launches0 = launch_count()
+    launches = 0
     wall0 = time.perf_counter()
-    for _ in range(args.steps):
-        flush.fill_(1)                      # evict L2 between timed steps
-        r.prepare_step()
+    for i in range(args.warmup, args.warmup + args.steps):
+        flush.fill_(1)                      # evict L2 between timed steps (outside the events)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        ev = []
-        e0.record()
-        r.step(ev)
-        e1.record()
+        if use_graph:
+            g = r.graph(i)
+            e0.record()
+            g.replay()
+            e1.record()
+            launches += g.kernels
+        else:
+            n0 = launch_count()
+            e0.record()
+            r.run(i)
+            e1.record()
+            launches += launch_count() - n0
         step_events.append((e0, e1))
-        evs.append(ev)
     barrier()
     wall = time.perf_counter() - wall0
-    launches = launch_count() - launches0
     clk = clocks.stop()
     step_ms = float(sum(a.elapsed_time(b) for a, b in step_events))
-    per_call = {}
-    for ev in evs:
-        for name, a, b in ev:
-            per_call.setdefault(name, []).append(a.elapsed_time(b))
     t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -350,23 +389,37 @@ def gpu_arm(args, wl):
     ms_per_step = step_ms / args.steps
     value = world * r.units_per_step / (ms_per_step / 1e3)
 
-    # e2e: pinned host inputs -> device, step, result -> host, all timed
-    e2e = e2e_leg(r, args, world, dev)
+    # per-call device time: each call alone, cold L2, queued behind a bounded sleep
+    per_call = {}
+    for i in range(args.warmup, args.warmup + min(args.steps, 5)):
+        for name, fn in r.calls(i):
+            flush.fill_(1)
+            torch.cuda._sleep(200000)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            per_call.setdefault(name, []).append((a, b))
+    torch.cuda.synchronize()
+    call_ms = {k: float(np.mean([a.elapsed_time(b) for a, b in v])) for k, v in per_call.items()}
+
+    e2e = e2e_leg(r, args, world, dev, use_graph)
 
     line = None
     if rank == 0:
         work = op_work(wl)
-        call_ms = {k: float(np.mean(v)) for k, v in per_call.items()}
         dom = max(call_ms, key=lambda k: call_ms[k])
         roof = roofline(dom, work[dom], call_ms[dom], peaks, peaks_src, wl)
         line = {
             "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) tokens/logits, E2M1 indexer codes, bf16 queries)",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
                        "H": wl.H, "D": wl.D, "HI": wl.HI, "dI": wl.dI,
                        "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                       "launch": "one CUDA graph per step" if use_graph else "direct C-ABI calls",
                        "parallelism": f"dp{world} (independent sequences per GPU)"},
             "roofline": roof,
             "per_call_ms": call_ms,
@@ -379,6 +432,8 @@ def gpu_arm(args, wl):
             line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     if world > 1:
         dist.barrier()
+    r.graphs.clear()
+    if world > 1:
         dist.destroy_process_group()
     return line
 
@@ -388,13 +443,12 @@ def launch_count():
     return csa.launch_count()
 
 
-def e2e_leg(r, args, world, dev):
-    """Same step through the public API with pinned host inputs copied in and the
-    attention output copied back inside the timed region."""
+def e2e_leg(r, args, world, dev, use_graph):
+    """The same step through the public API: pinned host inputs copied in and the
+    attention output copied back, all inside the timed region."""
     import torch
     wl = r.wl
-    if wl.kind in ("decode", "decode_incremental", "hca_decode"):
-        st = r.state
+    if r.decode:
         t0 = r.T0
         host = {"x": r.x[:, t0:t0 + r.n_new].contiguous().cpu().pin_memory(),
                 "z": r.z[:, t0:t0 + r.n_new].contiguous().cpu().pin_memory(),
@@ -402,28 +456,28 @@ def e2e_leg(r, args, world, dev):
         if wl.kind != "hca_decode":
             host["qI"] = r.ind.qI.cpu().pin_memory()
             host["w"] = r.ind.w.cpu().pin_memory()
-        out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
     else:
         host = {"x": r.x.cpu().pin_memory(), "z": r.z.cpu().pin_memory(), "q": r.q.cpu().pin_memory()}
-        out_host = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
+    out_dev = r.output()
+    out_host = torch.empty(out_dev.shape, dtype=out_dev.dtype).pin_memory()
     dbuf = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out_host.numel() * out_host.element_size()
-    saved_i = getattr(r, "step_i", None)
-    n = max(1, min(args.steps, 10))
+    step = args.warmup
+    g = r.graph(step, inputs=dbuf, key="e2e") if use_graph else None
     times = []
-    for i in range(n + 2):
-        if saved_i is not None and wl.kind == "decode_incremental":
-            r.step_i = saved_i
-        r.prepare_step()
+    for i in range(max(1, min(args.steps, 10)) + 2):
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
         for k in host:
             dbuf[k].copy_(host[k], non_blocking=True)
-        out = r.step(inputs=dbuf)
-        out_host.copy_(out, non_blocking=True)
+        if g is not None:
+            g.replay()
+        else:
+            r.run(step, inputs=dbuf)
+        out_host.copy_(out_dev, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
         if i >= 2:
@@ -616,6 +670,76 @@ def reference_arm(args, wl):
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def kernel_case(args, wl):
+    """One library call of the workload, alone, on inputs of the workload's
+    shape (no raw-token context): a small, repeatable target for profilers.
+    Cases: index_topk, attend, hca_attend, compress_entry."""
+    import torch
+
+    import compressed_sparse_attention_16_b200 as csa
+    import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, D, H, m, K, W = wl.B, wl.D, wl.H, wl.m, max(wl.K, 1), wl.W
+    decode = wl.kind != "prefill"
+    Tq = 1 if decode else wl.T
+    N = wl.N
+    q_pos = (torch.full((B, 1), wl.T - 1, dtype=torch.int32, device=dev) if decode
+             else torch.arange(wl.T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous())
+    d = csa.Dims(B=B, Tq=Tq, H=H, D=D, HI=max(wl.HI, 1), dI=max(wl.dI, 32), K=K, W=W, m=m, n_entries=N,
+                 entry_cap=N, win_cap=W if decode else wl.T)
+    case = args.kernel_case
+    if case == "index_topk":
+        ind = synth.indexer_inputs(B, Tq, N, wl.HI, wl.dI, 0, device=dev)
+        idx = torch.empty((B, Tq, K), dtype=torch.int32, device=dev)
+        sc = torch.empty((B, Tq, K), device=dev)
+        ws = torch.empty(max(1, csa.index_topk_workspace(d)), dtype=torch.uint8, device=dev)
+        fn = lambda: csa.index_topk(ind.qI, ind.w, ind.kI, q_pos, d, idx, sc, workspace=ws)
+    elif case in ("attend", "hca_attend"):
+        codes, scales = synth.e4m3_cache(B, N, D, 0, device=dev)
+        wcodes, wscales = synth.e4m3_cache(B, d.win_cap, D, 0, device=dev, tag="win")
+        q = synth.queries(B, Tq, H, D, wl.q_scale, 0, device=dev)
+        out = torch.empty((B, Tq, H, D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, Tq, H), device=dev)
+        dense = case == "hca_attend"
+        ws = torch.empty(max(1, csa.attend_workspace(d, dense)), dtype=torch.uint8, device=dev)
+        if dense:
+            fn = lambda: csa.hca_attend(q, codes, scales, wcodes, wscales, q_pos, d, out, lse, workspace=ws)
+        else:
+            g = torch.Generator(device=dev).manual_seed(0)
+            idx = torch.stack([torch.randperm(N, generator=g, device=dev)[:K] for _ in range(B * Tq)])
+            idx = idx.to(torch.int32).view(B, Tq, K).contiguous()
+            fn = lambda: csa.attend(q, codes, scales, idx, wcodes, wscales, q_pos, d, out, lse, workspace=ws)
+    elif case == "compress_entry":
+        n_tok = wl.m if wl.kind == "hca_decode" else (4 if decode else wl.T)
+        x, z = synth.tokens(B, n_tok, D, 0, device=dev)
+        codes = torch.empty((B, max(1, n_tok // m), D), dtype=torch.uint8, device=dev)
+        scales = torch.empty((B, max(1, n_tok // m)), device=dev)
+        fn = lambda: csa.compress(x, z, m, codes, scales)
+    else:
+        raise SystemExit(f"unknown kernel case {case}")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        torch.cuda._sleep(200000)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    csa.sync_status()
+    ms = [a.elapsed_time(b) for a, b in times]
+    print(json.dumps({"kernel_case": case, "workload": wl.name, "ms_mean": float(np.mean(ms)),
+                      "ms_min": float(np.min(ms)), "calls": args.steps,
+                      "device_bytes": int(torch.cuda.max_memory_allocated(dev))}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -625,9 +749,16 @@ def main():
     ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
+    ap.add_argument("--kernel-case", default=None,
+                    help="run one library call (index_topk, attend, hca_attend, compress_entry) alone on "
+                         "inputs of the workload's shape; for profilers")
     args = ap.parse_args()
     import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.kernel_case:
+        kernel_case(args, wl)
+        return
     if args.impl == "reference":
         line = reference_arm(args, wl)
     else:

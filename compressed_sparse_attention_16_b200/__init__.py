@@ -144,17 +144,21 @@ def _stream(stream) -> int | None:
 
 def compress(x: torch.Tensor, z: torch.Tensor, m: int, codes: torch.Tensor, scales: torch.Tensor,
              dst_first: int = 0, ring_cap: int = 0, pooled: torch.Tensor | None = None,
-             T: int | None = None, stream=None) -> None:
-    """csa_compress: pool full m-token blocks of x, z [B, Ttot, D] (first T tokens)
-    into codes u8 [B, cap, D] / scales f32 [B, cap] at slots dst_first + i."""
+             T: int | None = None, first_token: int = 0, stream=None) -> None:
+    """csa_compress: pool full m-token blocks of tokens [first_token, first_token + T)
+    of x, z [B, Ttot, D] into codes u8 [B, cap, D] / scales f32 [B, cap] at slots
+    dst_first + i (no copy of the token range is made)."""
     if x.dim() != 3 or z.shape != x.shape:
         raise ValueError("x and z must be [B, T, D] of equal shape")
     B, Ttot, D = x.shape
-    T = Ttot if T is None else T
+    T = Ttot - first_token if T is None else T
+    if first_token < 0 or first_token + T > Ttot:
+        raise ValueError("token range outside x")
     if codes.dim() != 3 or codes.shape[0] != B or codes.shape[2] != D or scales.shape != codes.shape[:2]:
         raise ValueError("codes must be [B, cap, D] and scales [B, cap]")
     dev = x.device
-    _check(lib().csa_compress(_ptr(x, torch.float32, "x"), _ptr(z, torch.float32, "z", dev),
+    off = first_token * D * 4
+    _check(lib().csa_compress(_ptr(x, torch.float32, "x") + off, _ptr(z, torch.float32, "z", dev) + off,
                               B, T, D, m, Ttot * D,
                               _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
                               dst_first, codes.shape[1], ring_cap,

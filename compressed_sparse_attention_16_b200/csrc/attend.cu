@@ -205,9 +205,7 @@ int launch_generic(const __nv_bfloat16 *q, const uint8_t *codes, const float *sc
   const int rows = d->B * d->Tq;
   const size_t smem = sizeof(float) * (kChunk * D + 8 * kChunk) + sizeof(void *) * kChunk +
                       sizeof(float) * kChunk + sizeof(int) * kMaxSel;
-  if (cudaFuncSetAttribute(attend_generic_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute(attend_generic_kernel)");
+  if (int rc = set_smem_once((const void *)attend_generic_kernel<D>, (int)smem, "attend_generic_kernel")) return rc;
   const dim3 grid((d->H + warps - 1) / warps, 1);
   // grid.y carries the row; split launches beyond 65535 rows
   for (int r0 = 0; r0 < rows; r0 += 65535) {
@@ -231,8 +229,15 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
                      const csa_dims *d, uint16_t *out, float *lse, void *workspace,
                      cudaStream_t stream);
 
-// 128 heads x 512-wide entries run on the tensor cores; other shapes use the
-// generic CUDA-core kernel above.
+bool attend_prefill_supported(const csa_dims *d);
+int launch_attend_prefill(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
+                          const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
+                          const csa_dims *d, uint16_t *out, float *lse, cudaStream_t stream);
+
+// 128 heads x 512-wide entries run on the tensor-core kernel with heads as
+// the MMA rows; 64 heads x 512 (selected entries + window <= 640 items) on the
+// one with items as the MMA rows; other shapes use the generic CUDA-core
+// kernel above.
 int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
                   const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
                   const csa_dims *d, uint16_t *out, float *lse, void *workspace, size_t ws_bytes,
@@ -241,6 +246,8 @@ int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, 
   if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
   if (attend_tc_supported(d))
     return launch_attend_tc(q, codes, scales, idx, wcodes, wscales, q_pos, d, out, lse, workspace, stream);
+  if (idx && attend_prefill_supported(d))
+    return launch_attend_prefill(q, codes, scales, idx, wcodes, wscales, q_pos, d, out, lse, stream);
   const auto *qb = reinterpret_cast<const __nv_bfloat16 *>(q);
   auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
   switch (d->D) {

@@ -502,8 +502,7 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
   a.ws_o = splits > 1 ? static_cast<float *>(workspace) : nullptr;
   a.ws_ml = splits > 1 ? reinterpret_cast<float2 *>(static_cast<char *>(workspace) + (size_t)(rows * splits * TH * TD * 4)) : nullptr;
   a.status = status_word_device_ptr();
-  if (cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute(attend_tc_kernel)");
+  if (int rc = set_smem_once((const void *)attend_tc_kernel, (int)SMEM_BYTES, "attend_tc_kernel")) return rc;
   const int64_t grid = rows * splits * 2;
   if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "attend: too many rows");
   attend_tc_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(a);

@@ -67,6 +67,24 @@ unsigned *status_word_device_ptr() {
   return ptrs[dev];
 }
 
+int set_smem_once(const void *kernel, int bytes, const char *name) {
+  static std::mutex mu;
+  static const void *done[64][16] = {{nullptr}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "%s: no device", name);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 16; ++i) {
+    if (done[dev][i] == kernel) return CSA_OK;
+    if (done[dev][i] == nullptr) {
+      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", name, cudaGetErrorString(e));
+      done[dev][i] = kernel;
+      return CSA_OK;
+    }
+  }
+  return fail(CSA_ERR_CUDA, "%s: attribute table full", name);
+}
+
 }  // namespace csa
 
 using namespace csa;

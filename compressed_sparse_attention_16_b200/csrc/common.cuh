@@ -29,6 +29,9 @@ enum : unsigned {
   STATUS_BAD_POSITION = 8u, // negative query position (treated as position 0 / no entries)
 };
 unsigned *status_word_device_ptr();   // address of the status word, current device
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel), so
+// that launches captured into CUDA graphs issue no attribute calls.
+int set_smem_once(const void *kernel, int bytes, const char *name);
 
 __device__ __forceinline__ void raise_status(unsigned *status, unsigned bit) {
   atomicOr(status, bit);

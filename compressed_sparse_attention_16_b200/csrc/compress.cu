@@ -124,6 +124,92 @@ compress_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_
   }
 }
 
+// Large blocks (m >= 16): one CTA per entry; G groups of D/4 threads each run
+// the online softmax over tokens g, g+G, g+2G, ... and the G partial states
+// (max, normaliser, weighted sum) are merged per channel in shared memory.
+__global__ void __launch_bounds__(1024)
+compress_tokens_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_per_seq,
+                       int D, int m, int G, int64_t x_bstride, uint8_t *__restrict__ codes,
+                       float *__restrict__ scales, int64_t dst_first, int64_t dst_bstride,
+                       int ring_cap, float *__restrict__ pooled) {
+  extern __shared__ float part[];            // [3][G][D]: max, normaliser, weighted sum
+  __shared__ float red[32];
+  const int L = D >> 2;
+  const int g = threadIdx.x / L, lane = threadIdx.x - g * L;
+  const int64_t e = blockIdx.x;
+  const int64_t b = e / n_per_seq, i = e - b * n_per_seq;
+  if (ring_cap > 0 && i + ring_cap < n_per_seq) return;     // overwritten later in this call
+  const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + lane;
+  const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + lane;
+  OnlineSoftmax4 sm;
+  sm.init();
+  int j = g;
+  for (; j + (kUnroll - 1) * G < m; j += kUnroll * G) {
+    float4 xv[kUnroll], zv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      xv[u] = __ldg(xp + (int64_t)(j + u * G) * L);
+      zv[u] = __ldg(zp + (int64_t)(j + u * G) * L);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) sm.push(xv[u], zv[u]);
+  }
+  for (; j < m; j += G) sm.push(__ldg(xp + (int64_t)j * L), __ldg(zp + (int64_t)j * L));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    part[(0 * G + g) * D + 4 * lane + c] = sm.mx[c];
+    part[(1 * G + g) * D + 4 * lane + c] = sm.l[c];
+    part[(2 * G + g) * D + 4 * lane + c] = sm.acc[c];
+  }
+  __syncthreads();
+  float C[4] = {0.f, 0.f, 0.f, 0.f};
+  float a = 0.f;
+  if (g == 0) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const int ch = 4 * lane + c;
+      float M = -INFINITY;
+      for (int k = 0; k < G; ++k) M = fmaxf(M, part[(0 * G + k) * D + ch]);
+      float l = 0.f, acc = 0.f;
+      for (int k = 0; k < G; ++k) {
+        const float mk = part[(0 * G + k) * D + ch];
+        if (mk == -INFINITY) continue;                  // a group that saw no token
+        const float f = expf(mk - M);
+        l = fmaf(part[(1 * G + k) * D + ch], f, l);
+        acc = fmaf(part[(2 * G + k) * D + ch], f, acc);
+      }
+      C[c] = __fdiv_rn(acc, l);
+    }
+    a = fmaxf(fmaxf(fabsf(C[0]), fabsf(C[1])), fmaxf(fabsf(C[2]), fabsf(C[3])));
+    const unsigned gm = L < 32 ? ((1u << L) - 1u) : 0xffffffffu;   // group 0's lanes of warp 0
+    for (int o = (L < 32 ? L : 32) >> 1; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(gm, a, o));
+    if (L > 32 && (threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+  }
+  __syncthreads();
+  if (g != 0) return;
+  if (L > 32) {
+    a = 0.f;
+    for (int k = 0; k < (L >> 5); ++k) a = fmaxf(a, red[k]);
+  }
+  float s = __fdiv_rn(a, 448.f);
+  if (!(s > 0.f)) s = 1.f;
+  uint32_t word = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t q = __nv_cvt_float_to_fp8(__fdiv_rn(C[c], s), __NV_SATFINITE, __NV_E4M3);
+    word |= q << (8 * c);
+  }
+  int64_t slot = dst_first + i;
+  if (ring_cap > 0) slot %= ring_cap;
+  const int64_t ent = b * dst_bstride + slot;
+  reinterpret_cast<uint32_t *>(codes + ent * D)[lane] = word;
+  if (lane == 0) scales[ent] = s;
+  if (pooled) {
+    reinterpret_cast<float4 *>(pooled + (b * n_per_seq + i) * (int64_t)D)[lane] =
+        make_float4(C[0], C[1], C[2], C[3]);
+  }
+}
+
 }  // namespace
 
 int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
@@ -133,6 +219,19 @@ int launch_compress(const float *x, const float *z, int B, int T, int D, int m, 
   const int64_t total = (int64_t)B * n;
   if (total == 0) return CSA_OK;
   const int L = D / 4;
+  if (m >= 16 && L <= 512) {
+    int G = 1024 / L;
+    while (G > 1 && G * 8 > m) G >>= 1;                 // at least 8 tokens per group
+    const size_t smem = (size_t)3 * G * D * sizeof(float);     // <= 3 * 1024 * 4 * 4 = 48 KiB
+    if (int rc = set_smem_once((const void *)compress_tokens_kernel, 3 * 1024 * 4 * 4, "compress_tokens_kernel"))
+      return rc;
+    if (total <= 0x7fffffffLL) {
+      compress_tokens_kernel<<<(unsigned)total, G * L, smem, stream>>>(
+          x, z, n, D, m, G, x_bstride, codes, scales, dst_first, dst_bstride, ring_cap, pooled);
+      count_launches(1);
+      return check_launch("compress_tokens_kernel");
+    }
+  }
   const int groups = kThreads / L;
   const int64_t grid = (total + groups - 1) / groups;
   if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");

@@ -22,6 +22,7 @@
 // the threshold are resolved by index, and the K survivors are sorted with a
 // bitonic network.
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace csa {
 namespace {
@@ -40,61 +41,56 @@ __device__ __forceinline__ int e2m1x2_int(uint32_t code) {   // 2*value of one 4
 constexpr int kScoreThreads = 256;
 constexpr int kEPT = 4;   // entries per thread per CTA
 
+// One query row of the indexer: 2*q as packed int8 (word 2k holds elements
+// 8k..8k+3, word 2k+1 elements 8k+4..8k+7) and 16*w as integers.
 template <int HI, int DI>
-__global__ void __launch_bounds__(kScoreThreads)
-index_scores_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
-                    const uint8_t *__restrict__ kI, const int32_t *__restrict__ q_pos, int row0,
-                    int Tq, int m, int n_entries, int64_t entry_cap, uint32_t *__restrict__ scores,
-                    int64_t ld, unsigned *status) {
-  constexpr int NW = DI / 8;           // 32-bit key words (8 codes each)
-  const int row = row0 + blockIdx.y;
-  const int b = row / Tq;
-  const int64_t t = q_pos[row];
-  const int nvis = (int)min((t + 1) / m, (int64_t)n_entries);
-  const int base = blockIdx.x * (kScoreThreads * kEPT);
-  if (base >= nvis) return;
-
-  // query as packed int8 (2*q): qw[h][2*k] holds elements 8k..8k+3, qw[h][2k+1] 8k+4..8k+7
+struct IndexQuery {
+  static constexpr int NW = DI / 8;     // 32-bit key words (8 codes each)
   int qw[HI][2 * NW];
   int w16[HI];
-  const uint8_t *qrow = qI + (int64_t)row * HI * (DI / 2);
+
+  __device__ __forceinline__ void load(const uint8_t *qrow, const float *wrow, unsigned *status,
+                                       bool report) {
 #pragma unroll
-  for (int h = 0; h < HI; ++h) {
-    const float wf = w[(int64_t)row * HI + h];
-    const float w16f = wf * 16.f;
-    w16[h] = __float2int_rn(w16f);
-    if (threadIdx.x == 0 && blockIdx.x == 0 && ((float)w16[h] != w16f || w16[h] < 0 || w16[h] > 16))
-      raise_status(status, STATUS_BAD_WEIGHT);
+    for (int h = 0; h < HI; ++h) {
+      const float w16f = wrow[h] * 16.f;
+      w16[h] = __float2int_rn(w16f);
+      if (report && ((float)w16[h] != w16f || w16[h] < 0 || w16[h] > 16)) raise_status(status, STATUS_BAD_WEIGHT);
 #pragma unroll
-    for (int k = 0; k < NW; ++k) {
-      const uint32_t word = *reinterpret_cast<const uint32_t *>(qrow + h * (DI / 2) + 4 * k);
-      uint32_t lo = 0, hi = 0;
+      for (int k = 0; k < NW; ++k) {
+        const uint32_t word = *reinterpret_cast<const uint32_t *>(qrow + h * (DI / 2) + 4 * k);
+        uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        lo |= (uint32_t)(e2m1x2_int((word >> (4 * e)) & 0xF) & 0xFF) << (8 * e);
-        hi |= (uint32_t)(e2m1x2_int((word >> (4 * e + 16)) & 0xF) & 0xFF) << (8 * e);
+        for (int e = 0; e < 4; ++e) {
+          lo |= (uint32_t)(e2m1x2_int((word >> (4 * e)) & 0xF) & 0xFF) << (8 * e);
+          hi |= (uint32_t)(e2m1x2_int((word >> (4 * e + 16)) & 0xF) & 0xFF) << (8 * e);
+        }
+        qw[h][2 * k] = (int)lo;
+        qw[h][2 * k + 1] = (int)hi;
       }
-      qw[h][2 * k] = (int)lo;
-      qw[h][2 * k + 1] = (int)hi;
     }
   }
 
-  const uint8_t *krow = kI + (int64_t)b * entry_cap * (DI / 2);
-  uint32_t *srow = scores + (int64_t)row * ld;
-#pragma unroll
-  for (int u = 0; u < kEPT; ++u) {
-    const int s = base + u * kScoreThreads + threadIdx.x;
-    if (s >= nvis) break;
-    uint32_t kw[NW];
+  __device__ __forceinline__ static void load_key(const uint8_t *krow, int64_t s, uint32_t (&kw)[NW]) {
     if constexpr (DI == 64) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4 *>(krow + (int64_t)s * 32));
-      const uint4 c = __ldg(reinterpret_cast<const uint4 *>(krow + (int64_t)s * 32 + 16));
+      const uint4 a = __ldg(reinterpret_cast<const uint4 *>(krow + s * 32));
+      const uint4 c = __ldg(reinterpret_cast<const uint4 *>(krow + s * 32 + 16));
       kw[0] = a.x; kw[1] = a.y; kw[2] = a.z; kw[3] = a.w;
       kw[4] = c.x; kw[5] = c.y; kw[6] = c.z; kw[7] = c.w;
     } else {
-      const uint4 a = __ldg(reinterpret_cast<const uint4 *>(krow + (int64_t)s * 16));
+      const uint4 a = __ldg(reinterpret_cast<const uint4 *>(krow + s * 16));
       kw[0] = a.x; kw[1] = a.y; kw[2] = a.z; kw[3] = a.w;
     }
+  }
+
+  // 64 * score of entry s (exact, < 2^24)
+  __device__ __forceinline__ uint32_t score(const uint8_t *krow, int64_t s) const {
+    uint32_t kw[NW];
+    load_key(krow, s, kw);
+    return score_words(kw);
+  }
+
+  __device__ __forceinline__ uint32_t score_words(const uint32_t (&kw)[NW]) const {
     int accP[HI], accN[HI];
 #pragma unroll
     for (int h = 0; h < HI; ++h) { accP[h] = 0; accN[h] = 0; }
@@ -117,7 +113,32 @@ index_scores_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
     uint32_t sc = 0;
 #pragma unroll
     for (int h = 0; h < HI; ++h) sc += (uint32_t)(w16[h] * max(accP[h] - accN[h], 0));
-    srow[s] = sc;
+    return sc;
+  }
+};
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(kScoreThreads)
+index_scores_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
+                    const uint8_t *__restrict__ kI, const int32_t *__restrict__ q_pos, int row0,
+                    int Tq, int m, int n_entries, int64_t entry_cap, uint32_t *__restrict__ scores,
+                    int64_t ld, unsigned *status) {
+  const int row = row0 + blockIdx.y;
+  const int b = row / Tq;
+  const int64_t t = q_pos[row];
+  const int nvis = (int)min((t + 1) / m, (int64_t)n_entries);
+  const int base = blockIdx.x * (kScoreThreads * kEPT);
+  if (base >= nvis) return;
+  IndexQuery<HI, DI> iq;
+  iq.load(qI + (int64_t)row * HI * (DI / 2), w + (int64_t)row * HI, status,
+          threadIdx.x == 0 && blockIdx.x == 0);
+  const uint8_t *krow = kI + (int64_t)b * entry_cap * (DI / 2);
+  uint32_t *srow = scores + (int64_t)row * ld;
+#pragma unroll
+  for (int u = 0; u < kEPT; ++u) {
+    const int s = base + u * kScoreThreads + threadIdx.x;
+    if (s >= nvis) break;
+    srow[s] = iq.score(krow, s);
   }
 }
 
@@ -211,23 +232,27 @@ __device__ void bitonic_asc_u32(uint32_t *a, int n) {
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-topk_rows_kernel(const uint32_t *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos,
-                 int m, int n_entries, int K, int32_t *__restrict__ idx_out,
-                 float *__restrict__ score_out, unsigned *status) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint64_t keys[kMaxK];
-  __shared__ uint32_t ties[kTieCap];
-  __shared__ uint32_t warp_tot[32];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above, s_cgt, s_ceq, s_run;
+struct RowSelSmem {
+  uint32_t hist[kBins];
+  uint64_t keys[kMaxK];
+  uint32_t ties[kTieCap];
+  uint32_t warp_tot[32];
+  int s_bin;
+  uint32_t s_above, s_cgt, s_ceq, s_run;
+};
 
-  const int row = blockIdx.x;
+// Exact top-K of the n scores S[0..n) (the entry index is the position), in
+// rank order, into out_idx[0..K) / out_score[0..K) (padding -1 / 0).
+// Called by all kSelThreads threads of a CTA.
+__device__ void select_row(const uint32_t *__restrict__ S, int n, int K, int32_t *__restrict__ out_idx,
+                           float *__restrict__ out_score, RowSelSmem &sm) {
+  uint32_t *hist = sm.hist;
+  uint64_t *keys = sm.keys;
+  uint32_t *ties = sm.ties;
+  uint32_t *warp_tot = sm.warp_tot;
+  int &s_bin = sm.s_bin;
+  uint32_t &s_above = sm.s_above, &s_cgt = sm.s_cgt, &s_ceq = sm.s_ceq, &s_run = sm.s_run;
   const int tid = threadIdx.x;
-  const int64_t t = q_pos[row];
-  if (t < 0 && tid == 0) raise_status(status, STATUS_BAD_POSITION);
-  const int n = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
-  const uint32_t *S = scores + (int64_t)row * ld;
   int cnt;
 
   if (n <= K) {
@@ -317,9 +342,22 @@ topk_rows_kernel(const uint32_t *__restrict__ scores, int64_t ld, const int32_t 
       id = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
       sc = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
     }
-    idx_out[(int64_t)row * K + j] = id;
-    if (score_out) score_out[(int64_t)row * K + j] = sc;
+    out_idx[j] = id;
+    if (out_score) out_score[j] = sc;
   }
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_rows_kernel(const uint32_t *__restrict__ scores, int64_t ld, const int32_t *__restrict__ q_pos,
+                 int m, int n_entries, int K, int32_t *__restrict__ idx_out,
+                 float *__restrict__ score_out, unsigned *status) {
+  __shared__ RowSelSmem sm;
+  const int row = blockIdx.x;
+  const int64_t t = q_pos[row];
+  if (t < 0 && threadIdx.x == 0) raise_status(status, STATUS_BAD_POSITION);
+  const int n = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  select_row(scores + (int64_t)row * ld, n, K, idx_out + (int64_t)row * K,
+             score_out ? score_out + (int64_t)row * K : nullptr, sm);
 }
 
 template <int HI, int DI>
@@ -335,9 +373,592 @@ void launch_scores(const uint8_t *qI, const float *w, const uint8_t *kI, const i
   }
 }
 
+// ---------------------------------------------------------------------------
+// split path for few query rows over many entries (decode): each CTA scores a
+// slice of entries and keeps its exact top-K as 64-bit keys; one CTA per row
+// then selects the final top-K among the slices' candidates.
+// ---------------------------------------------------------------------------
+constexpr int kPartThreads = 512;
+constexpr int kSliceMax = 8192;
+constexpr int kMergeThreads = 1024;
+constexpr int kMergeCap = 20480;     // candidate keys per row held by the merge CTA (160 KiB)
+
+// Bin (0..4095) where the count of keys in this-or-higher bins first reaches
+// `need`, and the count strictly above it.  NT threads, 4096/NT bins each.
+template <int NT>
+__device__ void find_bin(const uint32_t *hist, uint32_t need, uint32_t *warp_tot, int *out_bin,
+                         uint32_t *out_above) {
+  constexpr int BPT = kBins / NT;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hi_bin = kBins - 1 - BPT * tid;
+  uint32_t c[BPT], local = 0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) { c[k] = hist[hi_bin - k]; local += c[k]; }
+  uint32_t v = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += x;
+  }
+  if (lane == 31) warp_tot[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t wv = lane < NT / 32 ? warp_tot[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += x;
+    }
+    if (lane < NT / 32) warp_tot[lane] = wv;
+  }
+  __syncthreads();
+  const uint32_t incl = v + (warp > 0 ? warp_tot[warp - 1] : 0u);
+  const uint32_t excl = incl - local;
+  if (excl < need && incl >= need) {
+    uint32_t run = excl;
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+      if (run + c[k] >= need) { *out_bin = hi_bin - k; *out_above = run; break; }
+      run += c[k];
+    }
+  }
+  __syncthreads();
+}
+
+struct SelShared {
+  uint32_t warp_tot[32];
+  int bin;
+  uint32_t above;
+  uint32_t count;
+};
+
+// Threshold T such that exactly K of the n keys are >= T (keys distinct, K <= n):
+// radix select over the key bits, 12 bits per pass, stopping as soon as the
+// threshold bin is taken whole.
+template <int NT>
+__device__ uint64_t kth_largest_key(const uint64_t *keys, int n, int K, uint32_t *hist, SelShared *sh) {
+  uint64_t prefix = 0, pmask = 0;
+  uint32_t need = (uint32_t)K;
+  const int shifts[5] = {44, 32, 20, 8, 0};
+  const uint32_t dmask[5] = {0xFFFu, 0xFFFu, 0xFFFu, 0xFFFu, 0xFFu};
+  for (int dgt = 0; dgt < 5; ++dgt) {
+    const int sft = shifts[dgt];
+    const uint32_t dm = dmask[dgt];
+    for (int i = threadIdx.x; i < kBins; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int j = threadIdx.x; j < n; j += NT) {
+      const uint64_t k = keys[j];
+      if ((k & pmask) == prefix) atomicAdd(&hist[(uint32_t)(k >> sft) & dm], 1u);
+    }
+    __syncthreads();
+    find_bin<NT>(hist, need, sh->warp_tot, &sh->bin, &sh->above);
+    const uint32_t bin = (uint32_t)sh->bin;
+    need -= sh->above;
+    prefix |= (uint64_t)bin << sft;
+    pmask |= (uint64_t)dm << sft;
+    const uint32_t in_bin = hist[bin];
+    __syncthreads();
+    if (in_bin == need) break;       // the whole bin is taken: keys >= prefix
+  }
+  return prefix;
+}
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(kPartThreads)
+index_partial_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
+                     const uint8_t *__restrict__ kI, const int32_t *__restrict__ q_pos, int Tq, int m,
+                     int n_entries, int64_t entry_cap, int K, int splits, int slice,
+                     uint64_t *__restrict__ cand, unsigned *status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);                 // [kSliceMax]
+  uint32_t *hist = reinterpret_cast<uint32_t *>(keys + kSliceMax);         // [4096]
+  SelShared *sh = reinterpret_cast<SelShared *>(hist + kBins);
+  const int row = blockIdx.y, split = blockIdx.x, tid = threadIdx.x;
+  const int b = row / Tq;
+  int64_t t = q_pos[row];
+  if (t < 0) {
+    if (tid == 0 && split == 0) raise_status(status, STATUS_BAD_POSITION);
+    t = -1;
+  }
+  const int nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  const int s0 = split * slice;
+  const int n = max(0, min(s0 + slice, nvis) - s0);
+  uint64_t *out = cand + ((int64_t)row * splits + split) * K;
+  if (n == 0) {
+    for (int j = tid; j < K; j += kPartThreads) out[j] = 0ull;
+    return;
+  }
+  IndexQuery<HI, DI> iq;
+  iq.load(qI + (int64_t)row * HI * (DI / 2), w + (int64_t)row * HI, status, tid == 0 && split == 0);
+  const uint8_t *krow = kI + (int64_t)b * entry_cap * (DI / 2);
+  constexpr int U = 4;
+  for (int j0 = 0; j0 < n; j0 += kPartThreads * U) {
+    uint32_t kw[U][IndexQuery<HI, DI>::NW];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * kPartThreads + tid;
+      if (j < n) IndexQuery<HI, DI>::load_key(krow, s0 + j, kw[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * kPartThreads + tid;
+      if (j < n) keys[j] = make_key(iq.score_words(kw[u]), (uint32_t)(s0 + j));
+    }
+  }
+  __syncthreads();
+  if (n <= K) {
+    for (int j = tid; j < K; j += kPartThreads) out[j] = j < n ? keys[j] : 0ull;
+    return;
+  }
+  const uint64_t T = kth_largest_key<kPartThreads>(keys, n, K, hist, sh);
+  if (tid == 0) sh->count = 0;
+  __syncthreads();
+  for (int j = tid; j < n; j += kPartThreads) {
+    const uint64_t k = keys[j];
+    if (k >= T) out[atomicAdd(&sh->count, 1u)] = k;
+  }
+}
+
+__global__ void __launch_bounds__(kMergeThreads)
+topk_merge_kernel(const uint64_t *__restrict__ cand, int splits, int K, const int32_t *__restrict__ q_pos,
+                  int m, int n_entries, int32_t *__restrict__ idx_out, float *__restrict__ score_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);                 // [kMergeCap]
+  uint64_t *best = keys + kMergeCap;                                       // [kMaxK]
+  uint32_t *hist = reinterpret_cast<uint32_t *>(best + kMaxK);             // [4096]
+  SelShared *sh = reinterpret_cast<SelShared *>(hist + kBins);
+  const int row = blockIdx.x, tid = threadIdx.x;
+  const int64_t t = q_pos[row];
+  const int nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  const int n = splits * K;
+  const uint64_t *src = cand + (int64_t)row * n;
+  for (int j = tid; j < n; j += kMergeThreads) keys[j] = src[j];
+  if (tid == 0) sh->count = 0;
+  __syncthreads();
+  const int cnt = min(K, nvis);
+  // real candidates are non-zero keys; padding keys are 0 and rank last
+  const uint64_t T = (nvis > K) ? kth_largest_key<kMergeThreads>(keys, n, K, hist, sh) : 1ull;
+  for (int j = tid; j < n; j += kMergeThreads) {
+    const uint64_t k = keys[j];
+    if (k >= T) best[atomicAdd(&sh->count, 1u)] = k;
+  }
+  __syncthreads();
+  int np = 1;
+  while (np < cnt) np <<= 1;
+  for (int j = cnt + tid; j < np; j += kMergeThreads) best[j] = 0ull;
+  __syncthreads();
+  bitonic_desc_u64(best, np);
+  for (int j = tid; j < K; j += kMergeThreads) {
+    int32_t id = -1;
+    float sc = 0.f;
+    if (j < cnt) {
+      const uint64_t k = best[j];
+      id = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
+      sc = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
+    }
+    idx_out[(int64_t)row * K + j] = id;
+    if (score_out) score_out[(int64_t)row * K + j] = sc;
+  }
+}
+
+// Split-path plan: slices of at most kSliceMax entries, at most kMergeCap
+// candidates per row, about two CTAs per SM.  False when the row path applies.
+bool split_plan(const csa_dims *d, int *splits, int *slice) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  const int n = d->n_entries;
+  if (rows < 1 || rows > 64 || n < 2048) return false;
+  int s = (int)((2 * 148 + rows - 1) / rows);
+  s = min(s, (n + 1023) / 1024);
+  s = min(s, kMergeCap / d->K);
+  s = max(s, (n + kSliceMax - 1) / kSliceMax);
+  if (s * d->K > kMergeCap || s < 2) return false;
+  *splits = s;
+  *slice = (n + s - 1) / s;
+  return *slice <= kSliceMax;
+}
+
+template <int HI, int DI>
+void launch_partial(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+                    const csa_dims *d, int splits, int slice, uint64_t *cand, cudaStream_t stream) {
+  const size_t smem = kSliceMax * 8 + kBins * 4 + sizeof(SelShared);
+  if (set_smem_once((const void *)index_partial_kernel<HI, DI>, (int)smem, "index_partial_kernel")) return;
+  index_partial_kernel<HI, DI><<<dim3(splits, d->B * d->Tq), kPartThreads, smem, stream>>>(
+      qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, splits, slice, cand,
+      status_word_device_ptr());
+  count_launches(1);
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core decode path (dI = 64, HI <= 4, few query rows over many
+// entries).  Scores come from one block-scaled FP4 MMA per 128 keys
+// (kind::mxf4, M = 128 keys, N = 8 query rows = the heads padded with zeros,
+// K = 64, every scale 2^0).  The MMA's fp32 sums of E2M1 products are exact
+// (multiples of 1/4 below 2^12), so 4*acc is an integer and the score is
+// rebuilt in integers.
+//   scan:    keys stream HBM -> shared memory (cp.async, FP4 core-matrix
+//            layout); per 1024 keys 8 MMAs into TMEM; the epilogue writes each
+//            score to the workspace and counts it in a 4096-bin histogram of
+//            score >> 8, added into the row's global histogram.
+//   collect: every CTA derives the row's threshold bin (the bin holding the
+//            K-th best score) from the global histogram and appends the keys
+//            at or above it; the last CTA of the row (atomic ticket after a
+//            memory fence) ranks those candidates by counting, which yields
+//            the rank order directly.  If ties flood the threshold bin beyond
+//            the candidate buffer, it runs the exact radix select on the
+//            stored scores instead.
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 256;
+constexpr int kTileKeys = 128;
+constexpr int kBatchTiles = 8;
+constexpr int kBatchKeys = kTileKeys * kBatchTiles;      // 1024
+constexpr uint32_t kBatchBytes = kBatchKeys * 32;        // 32 KiB of packed keys
+constexpr int kStages = 3;                               // key batches in shared memory
+constexpr uint32_t kScanTmemCols = 256;                  // 3 x 64 accumulator + 8 scale columns
+constexpr uint32_t kColSFA = 192, kColSFB = 196;
+constexpr uint32_t kScanSmem = kStages * kBatchBytes + 256 + kBins * 4 + 256;   // ~113 KiB: at most 2 CTAs/SM
+constexpr int kCollectSpan = 32768;                      // scores read by one collect CTA
+constexpr int kCandCap = 2048;
+constexpr int kCollectThreads = kSelThreads;
+constexpr unsigned long long kScanWaitNs = 2000000000ull;
+
+struct TcWs {
+  uint32_t *scores;   // [rows][ld]
+  uint32_t *hist;     // [rows][4096]
+  uint64_t *cand;     // [rows][kCandCap]
+  uint32_t *ccount;   // [rows]
+  uint32_t *done;     // [rows] collect tickets
+  uint32_t *sdone;    // [rows] scan tickets
+  uint32_t *meta;     // [rows][2]: threshold bin, candidate count (written by the last scan CTA)
+};
+
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kScanThreads, 2)
+index_scan_tc_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
+                     const uint8_t *__restrict__ kI, const int32_t *__restrict__ q_pos, int Tq, int m,
+                     int n_entries, int64_t entry_cap, int K, int slice, TcWs ws, int64_t ld,
+                     unsigned *status) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char *kbuf = smem;                                          // [kStages][32 KiB]
+  unsigned char *qbuf = smem + kStages * kBatchBytes;                  // 8 rows x 32 B
+  uint32_t *hist = reinterpret_cast<uint32_t *>(qbuf + 256);           // [4096]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(hist + kBins);         // [kStages]
+  uint32_t *tptr = reinterpret_cast<uint32_t *>(bars + kStages);
+  int *abort_flag = reinterpret_cast<int *>(tptr + 1);
+  int *last_flag = abort_flag + 1;
+  SelShared *sel = reinterpret_cast<SelShared *>(abort_flag + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.y, split = blockIdx.x;
+  const int b = row / Tq;
+  const int64_t t = q_pos[row];
+  if (t < 0 && tid == 0 && split == 0) raise_status(status, STATUS_BAD_POSITION);
+  const int nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  const int s0 = split * slice;
+  const int s1 = min(s0 + slice, nvis);
+  const uint8_t *krow = kI + (int64_t)b * entry_cap * 32;
+  const int n = max(0, s1 - s0);
+  const int nb = (n + kBatchKeys - 1) / kBatchKeys;
+  auto load = [&](int bb) {
+    unsigned char *buf = kbuf + (bb % kStages) * kBatchBytes;
+    const int base = s0 + bb * kBatchKeys;
+    for (int c = tid; c < 2 * kBatchKeys; c += kScanThreads) {
+      const int r = c >> 1, h = c & 1;
+      const int s = base + r;
+      unsigned char *dst = buf + (r >> 7) * 4096 + ((r & 127) >> 3) * 256 + h * 128 + (r & 7) * 16;
+      const bool ok = s < s1;
+      tc::cp_async16(dst, ok ? (const void *)(krow + (int64_t)s * 32 + h * 16) : (const void *)krow, ok ? 16u : 0u);
+    }
+    tc::cp_async_commit();
+  };
+  // start the key stream before any set-up
+  for (int bb = 0; bb < kStages - 1; ++bb) {
+    if (bb < nb) load(bb); else tc::cp_async_commit();
+  }
+
+  if (warp == 0) tc::tmem_alloc(tptr, kScanTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) tc::mbar_init(&bars[i], 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = tid; i < kBins; i += kScanThreads) hist[i] = 0;
+  // query tile, FP4 core-matrix layout: row r, K-half c at c*128 + r*16 (rows >= HI are zero)
+  if (tid < 16) {
+    const int r = tid & 7, c = tid >> 3;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < HI) v = *reinterpret_cast<const uint4 *>(qI + ((int64_t)row * HI + r) * 32 + c * 16);
+    *reinterpret_cast<uint4 *>(qbuf + c * 128 + r * 16) = v;
+  }
+  int w16[HI];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) {
+    const float f = w[(int64_t)row * HI + h] * 16.f;
+    w16[h] = __float2int_rn(f);
+    if (tid == 0 && split == 0 && ((float)w16[h] != f || w16[h] < 0 || w16[h] > 16))
+      raise_status(status, STATUS_BAD_WEIGHT);
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *tptr;
+  if (warp < 4) {     // block scales = 2^0 (UE8M0 127) in every byte the MMA may read
+    const uint32_t ones[4] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kColSFA, ones);
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kColSFB, ones);
+    tc::tmem_wait_st();
+  }
+
+  const uint32_t idesc = tc::idesc_mxf4(128, 8);
+  for (int bb = 0; bb < nb; ++bb) {
+    tc::cp_async_wait<kStages - 2>();      // batch bb has landed (one group is committed per batch)
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const int stg = bb % kStages;
+    const uint32_t par = (uint32_t)(bb / kStages) & 1u;
+    if (tid == 0) {
+      const uint32_t buf = tc::smem_u32(kbuf + stg * kBatchBytes);
+      const uint64_t bd = tc::smem_desc(tc::smem_u32(qbuf), 128, 256);
+#pragma unroll
+      for (int i = 0; i < kBatchTiles; ++i)
+        tc::mma_mxf4_ss(tbase + stg * 64 + i * 8, tc::smem_desc(buf + i * 4096, 128, 256), bd, idesc,
+                        tbase + kColSFA, tbase + kColSFB, 0);
+      tc::mma_commit(&bars[stg]);
+    }
+    // bounded wait for the batch's MMAs
+    bool ok = tc::mbar_try_wait(&bars[stg], par);
+    if (!ok) {
+      const uint64_t t0 = gtimer();
+      uint32_t it = 0;
+      while (!(ok = tc::mbar_try_wait(&bars[stg], par))) {
+        if ((++it & 255u) == 0 && (*(volatile int *)abort_flag || gtimer() - t0 > kScanWaitNs)) {
+          if (!*(volatile int *)abort_flag) raise_status(status, STATUS_TIMEOUT);
+          *(volatile int *)abort_flag = 1;
+          break;
+        }
+      }
+    }
+    tc::fence_after_sync();
+    if (ok) {
+      const int q = warp & 3;
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int tile = (warp >> 2) * 4 + i4;
+        uint32_t acc[4];
+        tc::tmem_ld4(tbase + ((uint32_t)(q * 32) << 16) + stg * 64 + tile * 8, acc);
+        tc::tmem_wait_ld();
+        const int s = s0 + bb * kBatchKeys + tile * kTileKeys + q * 32 + lane;
+        if (s < s1) {
+          uint32_t sc = 0;
+#pragma unroll
+          for (int h = 0; h < HI; ++h)
+            sc += (uint32_t)(w16[h] * max(0, __float2int_rn(4.f * __uint_as_float(acc[h]))));
+          ws.scores[(int64_t)row * ld + s] = sc;
+          atomicAdd(&hist[sc >> 8], 1u);
+        }
+      }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (*(volatile int *)abort_flag) break;
+    if (bb + kStages - 1 < nb) load(bb + kStages - 1); else tc::cp_async_commit();
+  }
+  tc::cp_async_wait<0>();
+  for (int i = tid; i < kBins; i += kScanThreads) {
+    const uint32_t c = hist[i];
+    if (c) atomicAdd(&ws.hist[(int64_t)row * kBins + i], c);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tbase, kScanTmemCols);
+  // the row's last scan CTA derives the threshold bin from the complete histogram
+  __threadfence();
+  if (tid == 0) *last_flag = atomicAdd(&ws.sdone[row], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  uint32_t bstar = 0, C = (uint32_t)nvis;
+  if (nvis > K) {
+    // L2-coherent loads (not cached in L1), issued together
+    const uint4 *G = reinterpret_cast<const uint4 *>(ws.hist + (int64_t)row * kBins);
+    for (int i = tid; i < kBins / 4; i += kScanThreads) reinterpret_cast<uint4 *>(hist)[i] = __ldcg(G + i);
+    __syncthreads();
+    find_bin<kScanThreads>(hist, (uint32_t)K, sel->warp_tot, &sel->bin, &sel->above);
+    bstar = (uint32_t)sel->bin;
+    C = sel->above + hist[bstar];
+  }
+  if (tid == 0) {
+    ws.meta[2 * row] = bstar;
+    ws.meta[2 * row + 1] = C;
+  }
+}
+
+__global__ void __launch_bounds__(kCollectThreads)
+index_collect_kernel(const int32_t *__restrict__ q_pos, int m, int n_entries, int K, int span, TcWs ws,
+                     int64_t ld, int32_t *__restrict__ idx_out, float *__restrict__ score_out) {
+  __shared__ RowSelSmem sm;
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int row = blockIdx.y, split = blockIdx.x;
+  const int64_t t = q_pos[row];
+  const int nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  const uint32_t *S = ws.scores + (int64_t)row * ld;
+  uint32_t bstar = 0, C = (uint32_t)nvis;
+  if (nvis > 0) {
+    bstar = ws.meta[2 * row];
+    C = ws.meta[2 * row + 1];
+  }
+  const int slice = span;
+  const bool degenerate = C > (uint32_t)kCandCap;
+  if (!degenerate) {
+    // slice starts are multiples of 4 and rows are 16-byte aligned: read 4 scores at a time
+    const int j0 = split * slice;
+    const int j1 = min(j0 + slice, nvis);
+    uint64_t *cand = ws.cand + (int64_t)row * kCandCap;
+    const uint4 *S4 = reinterpret_cast<const uint4 *>(S + j0);
+    const int nq = (j1 - j0 + 3) >> 2;
+    constexpr int U = 4;
+    for (int q0 = 0; q0 < nq; q0 += kCollectThreads * U) {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int qi = q0 + u * kCollectThreads + tid;
+        v[u] = qi < nq ? __ldcg(S4 + qi) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int jb = j0 + 4 * (q0 + u * kCollectThreads + tid);
+        const uint32_t sv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = jb + e;
+          if (j < j1 && (sv[e] >> 8) >= bstar) {
+            const uint32_t pos = atomicAdd(&ws.ccount[row], 1u);
+            if (pos < (uint32_t)kCandCap) cand[pos] = make_key(sv[e], (uint32_t)j);
+          }
+        }
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&ws.done[row], 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int32_t *oi = idx_out + (int64_t)row * K;
+  float *os = score_out ? score_out + (int64_t)row * K : nullptr;
+  if (degenerate) {
+    select_row(S, nvis, K, oi, os, sm);
+    return;
+  }
+  const int cnt = min(K, nvis);
+  C = min(C, min(*(volatile uint32_t *)&ws.ccount[row], (uint32_t)kCandCap));
+  uint64_t *keys = sm.keys;                         // C <= kCandCap == kMaxK
+  const uint64_t *cand = ws.cand + (int64_t)row * kCandCap;
+  for (int i = tid; i < (int)C; i += kCollectThreads) keys[i] = *(volatile const uint64_t *)(cand + i);
+  __syncthreads();
+  // rank by counting: keys are distinct, so ranks are 0..C-1 in rank order
+  for (int i = tid; i < (int)C; i += kCollectThreads) {
+    const uint64_t k = keys[i];
+    int r = 0;
+    for (int j = 0; j < (int)C; ++j) r += keys[j] > k;
+    if (r < cnt) {
+      oi[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
+      if (os) os[r] = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
+    }
+  }
+  for (int j = cnt + tid; j < K; j += kCollectThreads) {
+    oi[j] = -1;
+    if (os) os[j] = 0.f;
+  }
+}
+
+// Tensor-core decode plan: about two CTAs per SM over the rows' entries.
+bool tc_plan(const csa_dims *d, int *splits, int *slice) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  const int n = d->n_entries;
+  if (d->dI != 64 || d->HI > 4 || rows < 1 || rows > 64 || n < 2048 || d->K > kMaxK) return false;
+  int s = (int)((2 * 148 + rows - 1) / rows);
+  s = min(s, (n + 1023) / 1024);
+  s = max(s, 1);
+  *splits = s;
+  *slice = (n + s - 1) / s;
+  return true;
+}
+
+size_t tc_workspace(const csa_dims *d, TcWs *ws, void *base) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
+  const size_t o_scores = take((size_t)(rows * ld * 4));
+  const size_t o_hist = take((size_t)(rows * kBins * 4));
+  const size_t o_cand = take((size_t)(rows * kCandCap * 8));
+  const size_t o_cnt = take((size_t)(rows * 4));
+  const size_t o_done = take((size_t)(rows * 4));
+  const size_t o_sdone = take((size_t)(rows * 4));
+  const size_t o_meta = take((size_t)(rows * 8));
+  if (ws && base) {
+    char *p = static_cast<char *>(base);
+    ws->scores = reinterpret_cast<uint32_t *>(p + o_scores);
+    ws->hist = reinterpret_cast<uint32_t *>(p + o_hist);
+    ws->cand = reinterpret_cast<uint64_t *>(p + o_cand);
+    ws->ccount = reinterpret_cast<uint32_t *>(p + o_cnt);
+    ws->done = reinterpret_cast<uint32_t *>(p + o_done);
+    ws->sdone = reinterpret_cast<uint32_t *>(p + o_sdone);
+    ws->meta = reinterpret_cast<uint32_t *>(p + o_meta);
+  }
+  return off;
+}
+
+int launch_tc(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+              const csa_dims *d, int splits, int slice, int32_t *idx_out, float *score_out,
+              void *workspace, cudaStream_t stream) {
+  TcWs ws;
+  tc_workspace(d, &ws, workspace);
+  const int rows = d->B * d->Tq;
+  const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
+  // the histogram and the counters start at zero on every call
+  const size_t zero_bytes = (size_t)((char *)ws.meta - (char *)ws.hist) + (size_t)rows * 8;
+  if (cudaMemsetAsync(ws.hist, 0, zero_bytes, stream) != cudaSuccess) return check_launch("cudaMemsetAsync");
+  if (int rc = set_smem_once((const void *)index_scan_tc_kernel<4>, (int)kScanSmem, "index_scan_tc_kernel")) return rc;
+  if (int rc = set_smem_once((const void *)index_scan_tc_kernel<2>, (int)kScanSmem, "index_scan_tc_kernel")) return rc;
+  if (int rc = set_smem_once((const void *)index_scan_tc_kernel<1>, (int)kScanSmem, "index_scan_tc_kernel")) return rc;
+  if (int rc = set_smem_once((const void *)index_scan_tc_kernel<3>, (int)kScanSmem, "index_scan_tc_kernel")) return rc;
+  const dim3 grid(splits, rows);
+  unsigned *st = status_word_device_ptr();
+  switch (d->HI) {
+    case 1: index_scan_tc_kernel<1><<<grid, kScanThreads, kScanSmem, stream>>>(qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, slice, ws, ld, st); break;
+    case 2: index_scan_tc_kernel<2><<<grid, kScanThreads, kScanSmem, stream>>>(qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, slice, ws, ld, st); break;
+    case 3: index_scan_tc_kernel<3><<<grid, kScanThreads, kScanSmem, stream>>>(qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, slice, ws, ld, st); break;
+    default: index_scan_tc_kernel<4><<<grid, kScanThreads, kScanSmem, stream>>>(qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, slice, ws, ld, st); break;
+  }
+  count_launches(1);
+  if (int rc = check_launch("index_scan_tc_kernel")) return rc;
+  const int csplits = (d->n_entries + kCollectSpan - 1) / kCollectSpan;
+  const int cspan = (((d->n_entries + csplits - 1) / csplits) + 3) & ~3;   // multiple of 4
+  index_collect_kernel<<<dim3(csplits, rows), kCollectThreads, 0, stream>>>(q_pos, d->m, d->n_entries, d->K, cspan,
+                                                                           ws, ld, idx_out, score_out);
+  count_launches(1);
+  return check_launch("index_collect_kernel");
+}
+
 }  // namespace
 
 size_t index_topk_workspace(const csa_dims *d) {
+  int splits, slice;
+  if (tc_plan(d, &splits, &slice)) return tc_workspace(d, nullptr, nullptr);
+  if (split_plan(d, &splits, &slice)) return (size_t)((int64_t)d->B * d->Tq * splits * d->K * 8);
   const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
   return (size_t)((int64_t)d->B * d->Tq * ld * 4);
 }
@@ -348,6 +969,28 @@ int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, cons
   const int rows = d->B * d->Tq;
   if (rows == 0) return CSA_OK;
   if (d->K > kMaxK) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: K > %d", kMaxK);
+  int splits, slice;
+  if (tc_plan(d, &splits, &slice))
+    return launch_tc(qI, w, kI, q_pos, d, splits, slice, idx_out, score_out, workspace, stream);
+  if (split_plan(d, &splits, &slice)) {
+    uint64_t *cand = static_cast<uint64_t *>(workspace);
+#define CSA_PARTIAL(HI_, DI_)                                                                   \
+  if (d->HI == HI_ && d->dI == DI_) {                                                           \
+    launch_partial<HI_, DI_>(qI, w, kI, q_pos, d, splits, slice, cand, stream);                 \
+  } else
+    CSA_PARTIAL(1, 32) CSA_PARTIAL(1, 64) CSA_PARTIAL(2, 32) CSA_PARTIAL(2, 64) CSA_PARTIAL(4, 32)
+    CSA_PARTIAL(4, 64) CSA_PARTIAL(8, 32) {
+      return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: (HI=%d, dI=%d) not compiled", d->HI, d->dI);
+    }
+#undef CSA_PARTIAL
+    if (int rc = check_launch("index_partial_kernel")) return rc;
+    const size_t smem = (kMergeCap + kMaxK) * 8 + kBins * 4 + sizeof(SelShared);
+    if (int rc = set_smem_once((const void *)topk_merge_kernel, (int)smem, "topk_merge_kernel")) return rc;
+    topk_merge_kernel<<<rows, kMergeThreads, smem, stream>>>(cand, splits, d->K, q_pos, d->m, d->n_entries,
+                                                             idx_out, score_out);
+    count_launches(1);
+    return check_launch("topk_merge_kernel");
+  }
   const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
   uint32_t *scores = static_cast<uint32_t *>(workspace);
   if (d->n_entries > 0) {

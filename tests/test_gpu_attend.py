@@ -68,6 +68,9 @@ CASES = [
     (1, 9, 64, 512, 4, 2100, 512, 128, 8400, 512 ** -0.5),
     (3, 4, 16, 256, 4, 700, 100, 50, 64, 0.1),
     (1, 6, 8, 128, 2, 400, 33, 7, 7, 0.2),
+    # 64 heads x 512 (items as MMA rows): partial tiles, -1 anywhere, window-only rows
+    (2, 6, 64, 512, 4, 300, 100, 50, 1200, 0.1),
+    (1, 3, 64, 512, 4, 600, 512, 128, 128, 512 ** -0.5),
 ]
 
 

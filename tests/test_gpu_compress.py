@@ -28,7 +28,8 @@ def _run(B, T, D, m, seed, ring_cap=0, dst_first=0, cap=None, scale=1.0):
 
 
 @pytest.mark.parametrize("B,T,D,m", [(1, 512, 64, 4), (2, 2051, 512, 4), (3, 777, 512, 1),
-                                     (2, 128 * 9 + 77, 512, 128), (1, 1000, 128, 7), (2, 64, 256, 4)])
+                                     (2, 128 * 9 + 77, 512, 128), (1, 1000, 128, 7), (2, 64, 256, 4),
+                                     (2, 700, 64, 32), (1, 300, 256, 16), (2, 600, 512, 17)])
 def test_compress_parity(B, T, D, m):
     x, z, codes, scales, pooled = _run(B, T, D, m, seed=B * 1000 + T + m)
     n = T // m
