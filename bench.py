@@ -682,10 +682,11 @@ def kernel_case(args, wl):
     torch.cuda.set_device(dev)
     B, D, H, m, K, W = wl.B, wl.D, wl.H, wl.m, max(wl.K, 1), wl.W
     decode = wl.kind != "prefill"
-    Tq = 1 if decode else wl.T
+    Tq = 1 if decode else (args.rows or wl.T)
     N = wl.N
+    # prefill: the last Tq positions of the sequence (the heaviest rows)
     q_pos = (torch.full((B, 1), wl.T - 1, dtype=torch.int32, device=dev) if decode
-             else torch.arange(wl.T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous())
+             else (wl.T - Tq + torch.arange(Tq, dtype=torch.int32, device=dev)).repeat(B, 1).contiguous())
     d = csa.Dims(B=B, Tq=Tq, H=H, D=D, HI=max(wl.HI, 1), dI=max(wl.dI, 32), K=K, W=W, m=m, n_entries=N,
                  entry_cap=N, win_cap=W if decode else wl.T)
     case = args.kernel_case
@@ -706,9 +707,11 @@ def kernel_case(args, wl):
         if dense:
             fn = lambda: csa.hca_attend(q, codes, scales, wcodes, wscales, q_pos, d, out, lse, workspace=ws)
         else:
+            # K distinct entries per row: a random offset plus a fixed random pattern of distinct steps
             g = torch.Generator(device=dev).manual_seed(0)
-            idx = torch.stack([torch.randperm(N, generator=g, device=dev)[:K] for _ in range(B * Tq)])
-            idx = idx.to(torch.int32).view(B, Tq, K).contiguous()
+            base = torch.randperm(N, generator=g, device=dev)[:K]
+            shift = torch.randint(0, N, (B * Tq, 1), generator=g, device=dev)
+            idx = ((base[None] + shift) % N).to(torch.int32).view(B, Tq, K).contiguous()
             fn = lambda: csa.attend(q, codes, scales, idx, wcodes, wscales, q_pos, d, out, lse, workspace=ws)
     elif case == "compress_entry":
         n_tok = wl.m if wl.kind == "hca_decode" else (4 if decode else wl.T)
@@ -750,6 +753,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
+    ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
                     help="run one library call (index_topk, attend, hca_attend, compress_entry) alone on "
                          "inputs of the workload's shape; for profilers")

@@ -224,40 +224,67 @@ __global__ void __launch_bounds__(kPThreads, 1) attend_prefill_kernel(const PArg
       tc::cp_async_commit();
     }
 
-    // gather + convert one 128-item x 128-d block into buffer `buf`
-    auto fill = [&](int tile, int dblk, int buf) {
+    // Block j of a pass covers items [tile*128, +128) and d [dblk*128, +128)
+    // with tile = j / 4, dblk = j % 4.  Its 16 KiB of E4M3 codes are gathered
+    // with cp.async into a staging ring that lives in shared memory the pass
+    // does not use (pass 1: the P^T region, 5 slots; pass 2: the Q region, 4
+    // slots), several blocks ahead; convert() turns a staged block into bf16
+    // tiles.  Staging layout [item][8 x 16 B], chunk c of item i at slot
+    // c ^ (i & 7) so that the conversion reads hit distinct banks.
+    constexpr uint32_t STG = PT * PDB;                  // 16 KiB per block
+    const int nblk_row = ntiles * (PD / PDB);
+    auto issue = [&](int pass, int j) {
+      if (j < nblk_row) {
+        const int tile = j / (PD / PDB), dblk = j % (PD / PDB);
+        const int nslot = pass == 0 ? 5 : 4;
+        unsigned char *st = smem + (pass == 0 ? P_OFF_PT : P_OFF_Q) + (j % nslot) * STG;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = tid + kPThreads * k;
+          const int item = c >> 3, ch = c & 7;
+          const int u = tile * PT + item;
+          const uint8_t *src = nullptr;
+          if (u < nsel) src = a.codes + ((int64_t)b * a.entry_cap + sel[u]) * PD;
+          else if (u < n_items) src = a.wcodes + ((int64_t)b * a.win_cap + ((p0 + (u - nsel)) % a.win_cap)) * PD;
+          tc::cp_async16(st + item * 128 + ((ch ^ (item & 7)) << 4),
+                         src ? (const void *)(src + dblk * PDB + ch * 16) : (const void *)a.codes, src ? 16u : 0u);
+        }
+      }
+      tc::cp_async_commit();
+    };
+    const int i8 = lane & 7, pq = lane >> 3;
+    auto convert = [&](int pass, int j, int buf) {
+      const int nslot = pass == 0 ? 5 : 4;
+      const unsigned char *st = smem + (pass == 0 ? P_OFF_PT : P_OFF_Q) + (j % nslot) * STG;
       unsigned char *kv = smem + P_OFF_KV + buf * P_KV_BYTES;
-      const int i8 = lane & 7, pq = lane >> 3;
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int item = (warp * 2 + r) * 8 + i8;        // 16 item groups over 8 warps
-        const int u = tile * PT + item;
-        const uint8_t *src = nullptr;
-        if (u < nsel) src = a.codes + ((int64_t)b * a.entry_cap + sel[u]) * PD;
-        else if (u < n_items) src = a.wcodes + ((int64_t)b * a.win_cap + ((p0 + (u - nsel)) % a.win_cap)) * PD;
-        uint4 c[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          c[k] = src ? __ldg(reinterpret_cast<const uint4 *>(src + dblk * PDB) + pq + 4 * k) : make_uint4(0, 0, 0, 0);
+        const int item = (warp * 2 + r) * 8 + i8;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           const int p = pq + 4 * k;                     // 16 codes -> d-groups 2p, 2p+1
+          const uint4 c = *reinterpret_cast<const uint4 *>(st + item * 128 + ((p ^ (item & 7)) << 4));
           uint4 lo, hi;
-          cvt16(c[k], lo, hi);
+          cvt16(c, lo, hi);
           *reinterpret_cast<uint4 *>(kv + pkv_off(item, 2 * p)) = lo;
           *reinterpret_cast<uint4 *>(kv + pkv_off(item, 2 * p + 1)) = hi;
         }
       }
       tc::fence_proxy_async_smem();
     };
+    constexpr int AHEAD1 = 4, AHEAD2 = 3;               // blocks in flight per pass
+
     // ---------------------------------------------------------------- pass 1
-    const int nblk = ntiles * (PD / PDB);
-    tc::cp_async_wait<0>();
+    const int nblk = nblk_row;
+    for (int j = 0; j < AHEAD1; ++j) issue(0, j);
     for (int j = 0; j < nblk && ok; ++j) {
       const int buf = j & 1;
       const int tile = j / (PD / PDB), dblk = j % (PD / PDB);
+      issue(0, j + AHEAD1);                              // into the slot block j-1 used
+      tc::cp_async_wait<AHEAD1>();                       // block j (and Q) have landed
+      __syncthreads();
       if (!drain(buf)) { ok = false; break; }
-      fill(tile, dblk, buf);
+      convert(0, j, buf);
       tc::fence_before_sync();
       __syncthreads();
       tc::fence_after_sync();
@@ -273,9 +300,12 @@ __global__ void __launch_bounds__(kPThreads, 1) attend_prefill_kernel(const PArg
       }
       issued[buf] += 1u;
     }
-    // all of pass 1 complete
+    // all of pass 1 complete; Q is no longer read, so pass 2 may stage into it
     if (ok) ok = drain(0) && drain(1);
     if (!ok) break;
+    tc::cp_async_wait<0>();
+    __syncthreads();
+    for (int j = 0; j < AHEAD2; ++j) issue(1, j);
     tc::fence_after_sync();
 
     // ---------------------------------------------------------------- softmax
@@ -339,8 +369,11 @@ __global__ void __launch_bounds__(kPThreads, 1) attend_prefill_kernel(const PArg
     for (int j = 0; j < nblk && ok; ++j) {
       const int buf = j & 1;
       const int tile = j / (PD / PDB), dblk = j % (PD / PDB);
+      issue(1, j + AHEAD2);
+      tc::cp_async_wait<AHEAD2>();
+      __syncthreads();
       if (!drain(buf)) { ok = false; break; }
-      fill(tile, dblk, buf);
+      convert(1, j, buf);
       tc::fence_before_sync();
       __syncthreads();
       tc::fence_after_sync();
@@ -358,6 +391,7 @@ __global__ void __launch_bounds__(kPThreads, 1) attend_prefill_kernel(const PArg
       }
       issued[buf] += 1u;
     }
+    tc::cp_async_wait<0>();
     if (ok) ok = drain(0) && drain(1);
     if (!ok) break;
     tc::fence_after_sync();

@@ -834,6 +834,7 @@ index_collect_kernel(const int32_t *__restrict__ q_pos, int m, int n_entries, in
         const int qi = q0 + u * kCollectThreads + tid;
         v[u] = qi < nq ? __ldcg(S4 + qi) : make_uint4(0, 0, 0, 0);
       }
+      const int lane = tid & 31;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int jb = j0 + 4 * (q0 + u * kCollectThreads + tid);
@@ -841,9 +842,18 @@ index_collect_kernel(const int32_t *__restrict__ q_pos, int m, int n_entries, in
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = jb + e;
-          if (j < j1 && (sv[e] >> 8) >= bstar) {
-            const uint32_t pos = atomicAdd(&ws.ccount[row], 1u);
-            if (pos < (uint32_t)kCandCap) cand[pos] = make_key(sv[e], (uint32_t)j);
+          const bool take = j < j1 && (sv[e] >> 8) >= bstar;
+          // one atomic per warp for all of its candidates
+          const unsigned msk = __ballot_sync(0xffffffffu, take);
+          if (msk) {
+            const int leader = __ffs(msk) - 1;
+            uint32_t base = 0;
+            if (lane == leader) base = atomicAdd(&ws.ccount[row], (uint32_t)__popc(msk));
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (take) {
+              const uint32_t pos = base + __popc(msk & ((1u << lane) - 1u));
+              if (pos < (uint32_t)kCandCap) cand[pos] = make_key(sv[e], (uint32_t)j);
+            }
           }
         }
       }
@@ -865,17 +875,16 @@ index_collect_kernel(const int32_t *__restrict__ q_pos, int m, int n_entries, in
   C = min(C, min(*(volatile uint32_t *)&ws.ccount[row], (uint32_t)kCandCap));
   uint64_t *keys = sm.keys;                         // C <= kCandCap == kMaxK
   const uint64_t *cand = ws.cand + (int64_t)row * kCandCap;
-  for (int i = tid; i < (int)C; i += kCollectThreads) keys[i] = *(volatile const uint64_t *)(cand + i);
+  int np = 1;
+  while (np < (int)C) np <<= 1;
+  for (int i = tid; i < np; i += kCollectThreads) keys[i] = i < (int)C ? __ldcg(cand + i) : 0ull;
   __syncthreads();
-  // rank by counting: keys are distinct, so ranks are 0..C-1 in rank order
-  for (int i = tid; i < (int)C; i += kCollectThreads) {
-    const uint64_t k = keys[i];
-    int r = 0;
-    for (int j = 0; j < (int)C; ++j) r += keys[j] > k;
-    if (r < cnt) {
-      oi[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
-      if (os) os[r] = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
-    }
+  // keys are distinct: after a descending sort the first cnt are the answer in rank order
+  bitonic_desc_u64(keys, np);
+  for (int r = tid; r < cnt; r += kCollectThreads) {
+    const uint64_t k = keys[r];
+    oi[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
+    if (os) os[r] = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
   }
   for (int j = cnt + tid; j < K; j += kCollectThreads) {
     oi[j] = -1;
@@ -953,11 +962,329 @@ int launch_tc(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_
   return check_launch("index_collect_kernel");
 }
 
+// ---------------------------------------------------------------------------
+// tensor-core prefill path: one CTA per 128 query rows (one TMEM lane per
+// query), streaming 16-entry key tiles.  Per tile and head one kind::mxf4 MMA
+// (M = 128 queries, N = 16 entries, K = 64) gives exact q.k sums; each
+// epilogue thread turns its query's 16 columns into integer scores and runs an
+// exact radix threshold over four streaming passes on a private 256-bin
+// histogram column (bits 19..12, 11..4, 3..0, then collection).  Entries are
+// visited in increasing index order, so the ties kept at the threshold are
+// the lowest-indexed ones.  Survivors are written in index order and put in
+// rank order by topk_sort_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kPfQ = 128;                 // queries per CTA
+constexpr int kPfN = 16;                  // entries per MMA tile
+constexpr int kPfStages = 8;              // key-tile ring
+constexpr int kPfThreads = 160;           // warps 0-3 epilogue, warp 4 control
+constexpr uint32_t kPfTmemCols = 256;     // 2 x (4 heads x 16) accumulator columns + scales
+constexpr uint32_t kPfColSFA = 128, kPfColSFB = 132;
+constexpr uint32_t kPfOffQ = 0;                                   // 4 heads x 4 KiB
+constexpr uint32_t kPfOffK = kPfOffQ + 4 * 4096;                  // stages x 512 B
+constexpr uint32_t kPfOffH = kPfOffK + kPfStages * 512;           // u16 [256 bins][128 queries]
+constexpr uint32_t kPfOffBar = kPfOffH + 256 * kPfQ * 2;
+constexpr uint32_t kPfSmem = kPfOffBar + 32 * 8 + 64;
+
+template <int HI>
+__global__ void __launch_bounds__(kPfThreads, 2)
+index_prefill_tc_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w,
+                        const uint8_t *__restrict__ kI, const int32_t *__restrict__ q_pos, int Tq, int m,
+                        int n_entries, int64_t entry_cap, int K, int tiles_per_seq, int ntiles,
+                        int32_t *__restrict__ idx_out, uint32_t *__restrict__ sc_out, unsigned *status) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  uint16_t *hist = reinterpret_cast<uint16_t *>(smem + kPfOffH);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kPfOffBar);
+  uint64_t *tfull = bars, *tempty = bars + 2, *sempty = bars + 4;      // [2], [2], [kPfStages]
+  uint32_t *tptr = reinterpret_cast<uint32_t *>(bars + 4 + kPfStages);
+  int *nvmax_s = reinterpret_cast<int *>(tptr + 1);
+  int *abort_flag = nvmax_s + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = ntiles - 1 - (int)blockIdx.x;          // the heaviest tiles first
+  const int seq = tile / tiles_per_seq;
+  const int q0 = (tile - seq * tiles_per_seq) * kPfQ;       // first query of the tile in its sequence
+  const int nq = min(kPfQ, Tq - q0);
+  const int64_t row0 = (int64_t)seq * Tq + q0;
+  const uint8_t *krow = kI + (int64_t)seq * entry_cap * 32;
+
+  // this thread's query (epilogue threads only)
+  int nvis = 0;
+  float w64[HI];            // 64 * w: with it, sum_h w64_h * max(acc_h, 0) is 64 * score, an exact fp32 integer
+#pragma unroll
+  for (int h = 0; h < HI; ++h) w64[h] = 0.f;
+  if (warp < 4 && tid < nq) {
+    const int64_t t = q_pos[row0 + tid];
+    if (t < 0) raise_status(status, STATUS_BAD_POSITION);
+    nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+#pragma unroll
+    for (int h = 0; h < HI; ++h) {
+      const float f = w[(row0 + tid) * HI + h] * 16.f;
+      const int w16 = __float2int_rn(f);
+      if ((float)w16 != f || w16 < 0 || w16 > 16) raise_status(status, STATUS_BAD_WEIGHT);
+      w64[h] = (float)(4 * w16);
+    }
+  }
+  if (tid == 0) { *nvmax_s = 0; *abort_flag = 0; }
+  if (warp == 4) tc::tmem_alloc(tptr, kPfTmemCols);
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) { tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4); }
+    for (int i = 0; i < kPfStages; ++i) tc::mbar_init(&sempty[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // query tiles (A operands), FP4 core-matrix layout; rows beyond the tile are zero
+  for (int c = tid; c < 4 * kPfQ * 2; c += kPfThreads) {
+    const int h = c / (kPfQ * 2), r = (c >> 1) % kPfQ, half = c & 1;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (h < HI && r < nq) v = *reinterpret_cast<const uint4 *>(qI + ((row0 + r) * HI + h) * 32 + half * 16);
+    *reinterpret_cast<uint4 *>(smem + kPfOffQ + h * 4096 + (r >> 3) * 256 + half * 128 + (r & 7) * 16) = v;
+  }
+  // histogram columns start at zero
+  for (int i = tid; i < 256 * kPfQ / 2; i += kPfThreads) reinterpret_cast<uint32_t *>(hist)[i] = 0u;
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp < 4 && nvis > 0) atomicMax(nvmax_s, nvis);
+  tc::fence_after_sync();
+  const uint32_t tbase = *tptr;
+  if (warp < 4) {
+    const uint32_t ones[4] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kPfColSFA, ones);
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kPfColSFB, ones);
+    tc::tmem_wait_st();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int nvmax = *nvmax_s;
+  const int npass = nvmax > K ? 4 : 1;
+  const int n_et = (nvmax + kPfN - 1) / kPfN;
+  const int total = npass * n_et;
+
+  auto bounded_wait = [&](uint64_t *bar, uint32_t par) -> bool {
+    if (tc::mbar_try_wait(bar, par)) return true;
+    const uint64_t t0 = gtimer();
+    uint32_t it = 0;
+    while (!tc::mbar_try_wait(bar, par)) {
+      if ((++it & 255u) == 0) {
+        if (*(volatile int *)abort_flag) return false;
+        if (gtimer() - t0 > kScanWaitNs) { *(volatile int *)abort_flag = 1; raise_status(status, STATUS_TIMEOUT); return false; }
+      }
+    }
+    return true;
+  };
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- control warp
+    const uint32_t idesc = tc::idesc_mxf4(128, kPfN);
+    auto load = [&](int i) {
+      const int stg = i % kPfStages;
+      const int et = i % n_et;
+      const int r = lane >> 1, half = lane & 1;           // 16 entries x 2 halves = 32 chunks
+      const int s = et * kPfN + r;
+      const bool okk = s < n_entries;
+      tc::cp_async16(smem + kPfOffK + stg * 512 + (r >> 3) * 256 + half * 128 + (r & 7) * 16,
+                     okk ? (const void *)(krow + (int64_t)s * 32 + half * 16) : (const void *)krow, okk ? 16u : 0u);
+    };
+    constexpr int LA = kPfStages - 1;
+    for (int i = 0; i < LA; ++i) { if (i < total) load(i); tc::cp_async_commit(); }
+    bool ok = true;
+    for (int i = 0; i < total && ok; ++i) {
+      // refill the stage of tile i-1 with tile i+LA once MMA(i-1) is done
+      const int nxt = i + LA;
+      if (nxt < total) {
+        if (nxt >= kPfStages) ok = bounded_wait(&sempty[nxt % kPfStages], (uint32_t)((nxt / kPfStages) - 1) & 1u);
+        if (ok) load(nxt);
+      }
+      tc::cp_async_commit();
+      tc::cp_async_wait<LA>();
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      const int buf = i & 1;
+      if (lane == 0 && ok) {
+        if (i >= 2) ok = bounded_wait(&tempty[buf], (uint32_t)((i >> 1) - 1) & 1u);
+        if (ok) {
+          tc::fence_after_sync();
+          const uint64_t bd = tc::smem_desc(tc::smem_u32(smem + kPfOffK + (i % kPfStages) * 512), 128, 256);
+#pragma unroll
+          for (int h = 0; h < HI; ++h)
+            tc::mma_mxf4_ss(tbase + buf * 64 + h * kPfN, tc::smem_desc(tc::smem_u32(smem + kPfOffQ + h * 4096), 128, 256),
+                            bd, idesc, tbase + kPfColSFA, tbase + kPfColSFB, 0);
+          tc::mma_commit(&tfull[buf]);
+          tc::mma_commit(&sempty[i % kPfStages]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    tc::cp_async_wait<0>();
+  } else {
+    // ---------------------------------------------------------------- epilogue: one query per thread
+    const bool active = tid < nq;
+    const bool radix = nvis > K;
+    uint32_t b1 = 0, b2 = 0, tau = 0, need_eq = 0, above = 0;
+    int cnt = 0;
+    uint32_t eq_taken = 0;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // this query's u16 counters: slot(tid) puts the 32 lanes of a warp in 32 different banks
+    uint16_t *hcol = hist + (lane * 2 + (warp & 1) + (warp >> 1) * 64);
+    auto find = [&](int nb, uint32_t need, uint32_t &above_out) -> uint32_t {
+      uint32_t cum = 0;
+      int bsel = 0;
+      for (int bn = nb - 1; bn >= 0; --bn) {
+        const uint32_t c = hcol[bn * kPfQ];
+        if (cum + c >= need) { bsel = bn; break; }
+        cum += c;
+      }
+      above_out = cum;
+      for (int bn = 0; bn < 256; ++bn) hcol[bn * kPfQ] = 0;
+      return (uint32_t)bsel;
+    };
+    bool ok = true;
+    for (int i = 0; i < total && ok; ++i) {
+      const int pass = npass == 4 ? i / n_et : 3;
+      const int et = i % n_et;
+      const int buf = i & 1;
+      ok = bounded_wait(&tfull[buf], (uint32_t)(i >> 1) & 1u);
+      tc::fence_after_sync();
+      // the 4 heads' 16 columns: 4 x 16 columns issued together, one wait
+      uint32_t r[4][16];
+#pragma unroll
+      for (int h = 0; h < HI; ++h)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                     : "=r"(r[h][0]), "=r"(r[h][1]), "=r"(r[h][2]), "=r"(r[h][3]), "=r"(r[h][4]), "=r"(r[h][5]),
+                       "=r"(r[h][6]), "=r"(r[h][7]), "=r"(r[h][8]), "=r"(r[h][9]), "=r"(r[h][10]), "=r"(r[h][11]),
+                       "=r"(r[h][12]), "=r"(r[h][13]), "=r"(r[h][14]), "=r"(r[h][15])
+                     : "r"(tbase + lane_off + buf * 64 + h * kPfN));
+      tc::tmem_wait_ld();
+      uint32_t sc[kPfN];
+#pragma unroll
+      for (int j = 0; j < kPfN; ++j) {
+        float f = 0.f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) f = fmaf(w64[h], fmaxf(__uint_as_float(r[h][j]), 0.f), f);
+        sc[j] = __float2uint_rz(f);          // exact: an integer below 2^20
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[buf]);
+      if (!active) continue;
+      const int s0 = et * kPfN;
+      if (pass == 0) {
+        if (radix)
+#pragma unroll
+          for (int j = 0; j < kPfN; ++j)
+            if (s0 + j < nvis) hcol[(sc[j] >> 12) * kPfQ] += 1;
+      } else if (pass == 1) {
+        if (radix)
+#pragma unroll
+          for (int j = 0; j < kPfN; ++j)
+            if (s0 + j < nvis && (sc[j] >> 12) == b1) hcol[((sc[j] >> 4) & 0xFF) * kPfQ] += 1;
+      } else if (pass == 2) {
+        if (radix)
+#pragma unroll
+          for (int j = 0; j < kPfN; ++j)
+            if (s0 + j < nvis && (sc[j] >> 4) == ((b1 << 8) | b2)) hcol[(sc[j] & 0xF) * kPfQ] += 1;
+      } else {
+        int32_t *oi = idx_out + (row0 + tid) * K;
+        uint32_t *os = sc_out + (row0 + tid) * K;
+#pragma unroll
+        for (int j = 0; j < kPfN; ++j) {
+          const int s = s0 + j;
+          if (s >= nvis) break;
+          bool take;
+          if (!radix) take = true;
+          else if (sc[j] > tau) take = true;
+          else if (sc[j] == tau && eq_taken < need_eq) { take = true; ++eq_taken; }
+          else take = false;
+          if (take) { oi[cnt] = s; os[cnt] = sc[j]; ++cnt; }
+        }
+      }
+      // pass boundaries: per-query thresholds
+      if (et == n_et - 1 && radix) {
+        uint32_t a;
+        if (pass == 0) { b1 = find(256, (uint32_t)K, a); above = a; }
+        else if (pass == 1) { b2 = find(256, (uint32_t)K - above, a); above += a; }
+        else if (pass == 2) {
+          const uint32_t b3 = find(16, (uint32_t)K - above, a);
+          above += a;
+          tau = (b1 << 12) | (b2 << 4) | b3;
+          need_eq = (uint32_t)K - above;
+        }
+      }
+    }
+    if (active) {
+      int32_t *oi = idx_out + (row0 + tid) * K;
+      uint32_t *os = sc_out + (row0 + tid) * K;
+      for (int j = cnt; j < K; ++j) { oi[j] = -1; os[j] = 0; }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 4) tc::tmem_dealloc(tbase, kPfTmemCols);
+}
+
+// Rank order for rows written in index order: sort (score desc, index asc).
+__global__ void __launch_bounds__(256)
+topk_sort_kernel(int K, int32_t *__restrict__ idx_out, const uint32_t *__restrict__ sc_in,
+                 float *__restrict__ score_out) {
+  __shared__ uint64_t keys[kMaxK];
+  const int64_t row = blockIdx.x;
+  int np = 1;
+  while (np < K) np <<= 1;
+  for (int j = threadIdx.x; j < np; j += 256) {
+    uint64_t k = 0;
+    if (j < K) {
+      const int32_t id = idx_out[row * K + j];
+      if (id >= 0) k = make_key(sc_in[row * K + j], (uint32_t)id);
+    }
+    keys[j] = k;
+  }
+  __syncthreads();
+  bitonic_desc_u64(keys, np);
+  for (int j = threadIdx.x; j < K; j += 256) {
+    const uint64_t k = keys[j];
+    idx_out[row * K + j] = k ? (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu)) : -1;
+    if (score_out) score_out[row * K + j] = k ? (float)(uint32_t)(k >> 32) * (1.f / 64.f) : 0.f;
+  }
+}
+
+bool prefill_tc_plan(const csa_dims *d) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  return d->dI == 64 && d->HI <= 4 && rows > 64 && d->n_entries <= 65535 && d->K <= kMaxK && d->n_entries >= 1;
+}
+
+int launch_prefill_tc(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos,
+                      const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
+                      cudaStream_t stream) {
+  const int tiles_per_seq = (d->Tq + kPfQ - 1) / kPfQ;
+  const int ntiles = d->B * tiles_per_seq;
+  uint32_t *sc = static_cast<uint32_t *>(workspace);
+  unsigned *st = status_word_device_ptr();
+#define CSA_PF(HI_)                                                                                  \
+  case HI_:                                                                                          \
+    if (int rc = set_smem_once((const void *)index_prefill_tc_kernel<HI_>, (int)kPfSmem, "index_prefill_tc_kernel")) \
+      return rc;                                                                                     \
+    index_prefill_tc_kernel<HI_><<<ntiles, kPfThreads, kPfSmem, stream>>>(                           \
+        qI, w, kI, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, tiles_per_seq, ntiles, idx_out, sc, st); \
+    break;
+  switch (d->HI) {
+    CSA_PF(1) CSA_PF(2) CSA_PF(3) CSA_PF(4)
+    default: return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d", d->HI);
+  }
+#undef CSA_PF
+  count_launches(1);
+  if (int rc = check_launch("index_prefill_tc_kernel")) return rc;
+  topk_sort_kernel<<<(unsigned)((int64_t)d->B * d->Tq), 256, 0, stream>>>(d->K, idx_out, sc, score_out);
+  count_launches(1);
+  return check_launch("topk_sort_kernel");
+}
+
 }  // namespace
 
 size_t index_topk_workspace(const csa_dims *d) {
   int splits, slice;
   if (tc_plan(d, &splits, &slice)) return tc_workspace(d, nullptr, nullptr);
+  if (prefill_tc_plan(d)) return (size_t)((int64_t)d->B * d->Tq * d->K * 4);
   if (split_plan(d, &splits, &slice)) return (size_t)((int64_t)d->B * d->Tq * splits * d->K * 8);
   const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
   return (size_t)((int64_t)d->B * d->Tq * ld * 4);
@@ -972,6 +1299,7 @@ int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, cons
   int splits, slice;
   if (tc_plan(d, &splits, &slice))
     return launch_tc(qI, w, kI, q_pos, d, splits, slice, idx_out, score_out, workspace, stream);
+  if (prefill_tc_plan(d)) return launch_prefill_tc(qI, w, kI, q_pos, d, idx_out, score_out, workspace, stream);
   if (split_plan(d, &splits, &slice)) {
     uint64_t *cand = static_cast<uint64_t *>(workspace);
 #define CSA_PARTIAL(HI_, DI_)                                                                   \

@@ -136,3 +136,27 @@ def test_negative_position_is_reported():
     with pytest.raises(csa.CsaError) as e:
         _gpu_topk(inp.qI, inp.w, inp.kI, torch.tensor([[-5, 10]], dtype=torch.int32), 4, 8, N)
     assert e.value.code == csa.CSA_ERR_INVALID
+
+
+def test_prefill_path_ties_and_large_k():
+    """Many query rows (the prefill path): keys from {0, 1} codes give massive
+    ties at the threshold; K = 2048 and a partial last tile of query rows."""
+    g = torch.Generator().manual_seed(2)
+    B, Tq, N, m = 2, 300, 3000, 4
+    codes = torch.randint(0, 2, (B, N, 64), generator=g, dtype=torch.uint8)
+    kI = (codes[..., 0::2] | (codes[..., 1::2] << 4)).contiguous()
+    inp = synth.indexer_inputs(B, Tq, 1, 4, 64, seed=12)
+    pos = torch.randint(0, 4 * N + 40, (B, Tq), generator=g, dtype=torch.int32)
+    pos[0, :5] = torch.tensor([0, 3, 4 * N - 1, 4 * 100, 4 * 2048], dtype=torch.int32)
+    for K in (100, 2048):
+        _compare(inp.qI, inp.w, kI, pos, m, K, N)
+
+
+def test_prefill_path_random_two_sequences():
+    B, Tq, N, m, K = 2, 257, 6000, 4, 512
+    inp = synth.indexer_inputs(B, Tq, N, 4, 64, seed=13)
+    g = torch.Generator().manual_seed(3)
+    pos = torch.randint(0, 4 * N + 10, (B, Tq), generator=g, dtype=torch.int32)
+    _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
+    inp2 = synth.indexer_inputs(B, Tq, N, 2, 64, seed=14)
+    _compare(inp2.qI, inp2.w, inp2.kI, pos, m, 64, N)
