@@ -148,3 +148,27 @@ def test_hca_decode_1m_full_size():
     out, lse = _run_gpu(q, codes, scales, None, wcodes, wscales, q_pos, d)
     ro, rl = ocsa.hca_attend(_bits(q), ent, lambda b, p: wv[b, p % W], q_pos, m, W)
     parity.check_attention(out, lse, ro, rl)
+
+
+@pytest.mark.parametrize("H", [64, 128, 16])
+@pytest.mark.parametrize("qexp,sexp", [((-16, -6), (-12, 12)), ((6, 10), (-30, -20))])
+def test_wide_dynamic_range(H, qexp, sexp):
+    """Per-head query magnitudes 2^qexp and per-entry scales 2^sexp / 448 far
+    from 1: the kernels that compute in fp16 bring both into range with exact
+    powers of two, which must not cost accuracy anywhere in these ranges."""
+    B, Tq, D, m, N, K, W, win_cap = 1, 5, 512, 4, 900, 512, 128, 128
+    rng = np.random.default_rng(H + qexp[0])
+    q_pos = rng.integers(0, m * N, (B, Tq)).astype(np.int32)
+    q_pos[0, 0] = 3
+    codes, _, wcodes, _, q, _, _ = _setup(B, Tq, H, D, N, win_cap, q_pos, 21, 1.0)
+    scales = torch.from_numpy((2.0 ** rng.uniform(*sexp, (B, N)) / 448.0).astype(np.float32))
+    wscales = torch.from_numpy((2.0 ** rng.uniform(*sexp, (B, win_cap)) / 448.0).astype(np.float32))
+    hf = torch.from_numpy(2.0 ** rng.integers(qexp[0], qexp[1] + 1, H).astype(np.float32))
+    q = (q.float() * hf[None, None, :, None]).to(torch.bfloat16)
+    ent = ocsa.dequantize(codes.numpy(), scales.numpy())
+    wv = ocsa.dequantize(wcodes.numpy(), wscales.numpy())
+    idx = _random_selection(rng, q_pos, m, N, K)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=win_cap, softmax_scale=D ** -0.5)
+    out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % win_cap], q_pos, W, scale=D ** -0.5)
+    parity.check_attention(out, lse, ro, rl)
