@@ -322,6 +322,15 @@ class Runner:
         return g
 
 
+def l2_flush(buf):
+    """Evict the L2 between timed steps: write a buffer larger than the L2, then
+    read it back, so the write-backs of the dirty lines also happen here and
+    not inside the next timed region."""
+    import torch
+    buf.fill_(1)
+    buf.view(torch.int64).sum()
+
+
 def gpu_arm(args, wl):
     import torch
     import torch.distributed as dist
@@ -362,7 +371,7 @@ def gpu_arm(args, wl):
     launches = 0
     wall0 = time.perf_counter()
     for i in range(args.warmup, args.warmup + args.steps):
-        flush.fill_(1)                      # evict L2 between timed steps (outside the events)
+        l2_flush(flush)                     # evict L2 between timed steps (outside the events)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         if use_graph:
@@ -393,7 +402,7 @@ def gpu_arm(args, wl):
     per_call = {}
     for i in range(args.warmup, args.warmup + min(args.steps, 5)):
         for name, fn in r.calls(i):
-            flush.fill_(1)
+            l2_flush(flush)
             torch.cuda._sleep(200000)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
@@ -418,7 +427,7 @@ def gpu_arm(args, wl):
             "data": "synthetic (seeded N(0,1) tokens/logits, E2M1 indexer codes, bf16 queries)",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
                        "H": wl.H, "D": wl.D, "HI": wl.HI, "dI": wl.dI,
-                       "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+                       "l2": "flushed between timed steps (256 MiB write then read, outside the step events)",
                        "launch": "one CUDA graph per step" if use_graph else "direct C-ABI calls",
                        "parallelism": f"dp{world} (independent sequences per GPU)"},
             "roofline": roof,
@@ -727,7 +736,7 @@ def kernel_case(args, wl):
     torch.cuda.synchronize()
     times = []
     for _ in range(args.steps):
-        flush.fill_(1)
+        l2_flush(flush)
         torch.cuda._sleep(200000)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)

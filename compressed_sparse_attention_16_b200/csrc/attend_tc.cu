@@ -9,17 +9,23 @@
 // window covers the latest 128 tokens.  The same key/value row serves as key
 // and as value, so one shared-memory tile feeds both products.
 //
-// Work split: one CTA per (query row, item split, half of D).  With M = 128
+// Work split: one CTA per (query row, half of D, item split).  With M = 128
 // query heads, S = Q K^T (K = 512) lands in TMEM with one head per lane; the
 // output half O[:, dh*256 : dh*256+256] = P V accumulates in 256 TMEM columns
-// across the CTA's chunks of 32 items.  Both CTAs of a row compute the same S
-// (each needs the full 512-wide dot products) and keep bit-identical softmax
-// state, so their halves combine without exchange.
+// across the CTA's chunks of 32 items.  Both halves of a row compute the same
+// S (each needs the full 512-wide dot products) and keep bit-identical softmax
+// state, so their halves combine without exchange.  The item splits of one
+// (row, half) (1, 2, 4 or 8) form a thread-block cluster: each CTA parks its
+// unnormalised partial O and per-head (max, sum) in its own shared memory and
+// the CTAs merge them through distributed shared memory, each producing the
+// final rows of 128 / splits heads:
+//   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
 //
 // Roles (288 threads):
 //   warps 0-3  gather 32 items per chunk, convert E4M3 codes exactly to bf16
 //              and store them in the "core matrix" layout (8 rows x 16 B);
-//   warps 4-7  softmax: one head per thread, lazy rescaling of O (only when a
+//   warps 4-7  Q to shared memory (while the first chunks are gathered), then
+//              softmax: one head per thread, lazy rescaling of O (only when a
 //              chunk raises the running max by more than 2^8), P = p * scale
 //              written to shared memory;
 //   warp 8     TMEM allocation and the single MMA-issuing thread.
@@ -59,7 +65,8 @@ constexpr uint32_t TCOL_O = 0;        // 256 columns
 constexpr uint32_t TCOL_S = 256;      // 2 x 32 columns
 constexpr uint32_t TMEM_COLS = 512;
 
-enum { BAR_KV_FULL = 0, BAR_KV_FREE = 2, BAR_S_FULL = 4, BAR_P_FULL = 6, BAR_PV_DONE = 8, BAR_FIN = 9 };
+enum { BAR_KV_FULL = 0, BAR_KV_FREE = 2, BAR_S_FULL = 4, BAR_P_FULL = 6, BAR_PV_DONE = 8, BAR_FIN = 9,
+       BAR_MREADY = 10, BAR_MDONE = 11, BAR_Q = 12 };
 
 struct Misc {
   uint32_t tmem_base;
@@ -91,6 +98,63 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc *m
   }
   return true;
 }
+
+// ---- cluster helpers (distributed shared memory)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void peer_arrive(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+__device__ __forceinline__ bool try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(tc::smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (acquire at cluster scope) for the first phase of `bar`.
+__device__ __forceinline__ bool wait_cluster_bar(uint64_t *bar, unsigned *status) {
+  const uint64_t t0 = globaltimer();
+  uint32_t n = 0;
+  while (!try_wait_cluster(bar, 0)) {
+    if ((++n & 255u) == 0 && globaltimer() - t0 > kWaitNs) {
+      raise_status(status, STATUS_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float2 ld_peer_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+  return v;
+}
+
+// Partial O in shared memory for the cluster merge: fp32 [128 heads][256 d]
+// over the Q region, 16-byte chunk c of head h at chunk c ^ (h & 7) (the
+// eight heads of a store phase hit distinct banks); (max, sum) per head in
+// the selection region.
+__device__ __forceinline__ uint32_t po_off(int h, int c) { return (uint32_t)h * 1024 + ((c ^ (h & 7)) << 4); }
 
 // Byte offsets in the core-matrix layouts.  g counts 16-byte groups along
 // the contraction-side dimension of each tile (8 bf16).  Every tile keeps
@@ -134,8 +198,6 @@ struct Args {
   int splits, cps;          // splits per row, chunks per split
   __nv_bfloat16 *out;
   float *lse;
-  float *ws_o;              // [rows, splits, 128, 512] partial outputs (splits > 1)
-  float2 *ws_ml;            // [rows, splits, 128] (max, sum) in log2 units
   unsigned *status;
 };
 
@@ -147,10 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
   float *iscale = reinterpret_cast<float *>(smem + OFF_SCALE);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int dh = blockIdx.x & 1;
-  const int rs = blockIdx.x >> 1;
-  const int split = rs % a.splits;
-  const int row = rs / a.splits;
+  const int split = blockIdx.x % a.splits;        // == rank in the cluster
+  const int pair = blockIdx.x / a.splits;
+  const int dh = pair & 1;
+  const int row = pair >> 1;
   const int b = row / a.Tq;
 
   int64_t t = a.q_pos[row];
@@ -166,7 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
     misc->abort = 0;
     for (int i = 0; i < 10; ++i) tc::mbar_init(&bars[i], (i == BAR_KV_FULL || i == BAR_KV_FULL + 1) ? 128
                                                        : (i == BAR_P_FULL || i == BAR_P_FULL + 1) ? 128 : 1);
+    tc::mbar_init(&bars[BAR_MREADY], (uint32_t)a.splits);
+    tc::mbar_init(&bars[BAR_MDONE], (uint32_t)a.splits);
+    tc::mbar_init(&bars[BAR_Q], 128);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (a.splits > 1) {
+    // every CTA of the cluster has initialised its barriers before any remote arrival
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   }
   if (warp == 8) tc::tmem_alloc(&misc->tmem_base, TMEM_COLS);
 
@@ -199,20 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
   const int c_end = min(c_begin + a.cps, nch);
   const int nloc = max(0, c_end - c_begin);
 
-  // Q -> shared memory (warps 0-7), core-matrix layout
-  if (warp < 8 && nloc > 0) {
-    const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * TH * TD);
-    for (int it = 0; it < (TH * TD / 8) / 256; ++it) {
-      // lane pairs read 32 contiguous bytes of one head; a warp covers 16 heads
-      // idx bits: [0] g_lo, [1..4] h_lo, [5..7] h_hi, [8..12] g_hi
-      const int idx = it * 256 + tid;
-      const int h = ((idx >> 5) & 7) * 16 + ((idx >> 1) & 15);
-      const int g = (idx >> 8) * 2 + (idx & 1);
-      const uint4 v = __ldg(qrow + h * (TD / 8) + g);
-      *reinterpret_cast<uint4 *>(smem + OFF_Q + q_off(h, g)) = v;
-    }
-    tc::fence_proxy_async_smem();
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -259,6 +314,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
+    // Q -> shared memory (core-matrix layout) while the loaders gather the
+    // first chunks; lane pairs read 32 contiguous bytes of one head, a warp
+    // covers 16 heads; 8 loads in flight per thread
+    if (nloc > 0) {
+      const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * TH * TD);
+      const int t = tid - 128;
+#pragma unroll 1
+      for (int it0 = 0; it0 < (TH * TD / 8) / 128; it0 += 8) {
+        uint4 v[8];
+        int hh[8], gg[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          // idx bits: [0] g_lo, [1..4] h_lo, [5..6] h_hi, [7..12] g_hi
+          const int idx = (it0 + u) * 128 + t;
+          hh[u] = ((idx >> 5) & 3) * 16 + ((idx >> 1) & 15) + 64 * ((idx >> 7) & 1);
+          gg[u] = (idx >> 8) * 2 + (idx & 1);
+          v[u] = __ldg(qrow + hh[u] * (TD / 8) + gg[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(smem + OFF_Q + q_off(hh[u], gg[u])) = v[u];
+      }
+      tc::fence_proxy_async_smem();
+    }
+    tc::mbar_arrive(&bars[BAR_Q]);
     const int quad = warp - 4;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -323,22 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
     }
     // epilogue
     const int64_t orow = (int64_t)row * TH + h;
-    if (nloc == 0) {
-      if (a.splits > 1) {
-        if (dh == 0) a.ws_ml[((int64_t)row * a.splits + split) * TH + h] = make_float2(-INFINITY, 0.f);
-        float4 *dst = reinterpret_cast<float4 *>(a.ws_o + (((int64_t)row * a.splits + split) * TH + h) * TD + dh * DHALF);
-        for (int k = 0; k < DHALF / 4; ++k) dst[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    } else if (ok && wait_bar(&bars[BAR_PV_DONE], (nloc - 1) & 1, misc, a.status)) {
-      tc::fence_after_sync();
-      const bool final_out = a.splits == 1;
-      const float inv = 1.f / l;
+    const bool have = nloc > 0 && ok && wait_bar(&bars[BAR_PV_DONE], (nloc - 1) & 1, misc, a.status);
+    tc::fence_after_sync();
+    if (a.splits == 1) {
+      if (have) {
+        const float inv = 1.f / l;
 #pragma unroll 1
-      for (int blk = 0; blk < DHALF / 32; ++blk) {
-        uint32_t o[32];
-        tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
-        tc::tmem_wait_ld();
-        if (final_out) {
+        for (int blk = 0; blk < DHALF / 32; ++blk) {
+          uint32_t o[32];
+          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
+          tc::tmem_wait_ld();
           uint32_t w[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
@@ -348,21 +421,32 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
           uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * TD + dh * DHALF + blk * 32);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-        } else {
-          float4 *dst = reinterpret_cast<float4 *>(a.ws_o + (((int64_t)row * a.splits + split) * TH + h) * TD + dh * DHALF + blk * 32);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
         }
-      }
-      if (final_out) {
         if (a.lse && dh == 0) a.lse[orow] = (m_used + log2f(l)) * 0.6931471805599453f;
-      } else if (dh == 0) {
-        a.ws_ml[((int64_t)row * a.splits + split) * TH + h] = make_float2(m_used, l);
       }
+    } else {
+      // park the partial (zeros when this split had no items) for the merge;
+      // the Q tile is no longer read once the last PV has completed
+#pragma unroll 1
+      for (int blk = 0; blk < DHALF / 32; ++blk) {
+        uint32_t o[32];
+        if (have) {
+          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
+          tc::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          *reinterpret_cast<uint4 *>(smem + OFF_Q + po_off(h, blk * 8 + k)) =
+              make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+      }
+      reinterpret_cast<float2 *>(smem + OFF_SEL)[h] = have ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
+      asm volatile("fence.acq_rel.cluster;" ::: "memory");   // visible to the peers' reads
     }
   } else {
+    // ------------------------------------------------------------ MMA issuer  } else {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nloc > 0) {
       const uint32_t idesc_qk = tc::idesc_bf16_f32(128, CH, 0, 0);
@@ -379,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
         }
         tc::mma_commit(&bars[BAR_S_FULL + buf]);
       };
-      bool ok = wait_bar(&bars[BAR_KV_FULL + 0], 0, misc, a.status);
+      bool ok = wait_bar(&bars[BAR_Q], 0, misc, a.status) && wait_bar(&bars[BAR_KV_FULL + 0], 0, misc, a.status);
       if (ok) { tc::fence_after_sync(); issue_qk(0); }
       if (ok && nloc > 1) {
         ok = wait_bar(&bars[BAR_KV_FULL + 1], 0, misc, a.status);
@@ -417,75 +501,93 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 8) tc::tmem_dealloc(tbase, TMEM_COLS);
-}
 
-// Combine split partials: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void __launch_bounds__(256)
-attend_merge_kernel(const float *__restrict__ ws_o, const float2 *__restrict__ ws_ml, int splits,
-                    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
-  const int row = blockIdx.x;
-  const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, ws_ml[((int64_t)row * splits + s) * TH + h].x);
-  float L = 0.f;
-  float acc[16];
+  if (a.splits > 1) {
+    // ---- cluster merge: heads [rank * 128 / S, +128 / S) of this (row, half)
+    const uint32_t S = (uint32_t)a.splits;
+    const uint32_t rank = cluster_rank();
+    if (tid == 0)
+      for (uint32_t r = 0; r < S; ++r) peer_arrive(peer_addr(tc::smem_u32(&bars[BAR_MREADY]), r));
+    const bool ready = wait_cluster_bar(&bars[BAR_MREADY], a.status);
+    if (ready && warp < 8) {
+      const int hper = TH / (int)S;
+      for (int hh = warp; hh < hper; hh += 8) {
+        const int h = (int)rank * hper + hh;
+        // (max, sum) of source split `lane`
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (lane < (int)S) ml = ld_peer_f2(peer_addr(tc::smem_u32(smem + OFF_SEL) + h * 8, (uint32_t)lane));
+        float M = ml.x;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = ws_ml[((int64_t)row * splits + s) * TH + h];
-    if (ml.y == 0.f) continue;
-    const float wgt = exp2f(ml.x - M);
-    L += wgt * ml.y;
-    const float4 *src = reinterpret_cast<const float4 *>(ws_o + (((int64_t)row * splits + s) * TH + h) * TD) + lane * 4;
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float wgt = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
+        float L = wgt * ml.y;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 v = src[k];
-      acc[4 * k] += wgt * v.x; acc[4 * k + 1] += wgt * v.y;
-      acc[4 * k + 2] += wgt * v.z; acc[4 * k + 3] += wgt * v.w;
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        // all sources' loads in flight before any use
+        float wj[8];
+        float4 v0[8], v1[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          wj[j] = __shfl_sync(0xffffffffu, wgt, j);
+          v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (j < (int)S && wj[j] != 0.f) {
+            const uint32_t base = peer_addr(tc::smem_u32(smem + OFF_Q), (uint32_t)j);
+            v0[j] = ld_peer_f4(base + po_off(h, 2 * lane));
+            v1[j] = ld_peer_f4(base + po_off(h, 2 * lane + 1));
+          }
+        }
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc[0] += wj[j] * v0[j].x; acc[1] += wj[j] * v0[j].y; acc[2] += wj[j] * v0[j].z; acc[3] += wj[j] * v0[j].w;
+          acc[4] += wj[j] * v1[j].x; acc[5] += wj[j] * v1[j].y; acc[6] += wj[j] * v1[j].z; acc[7] += wj[j] * v1[j].w;
+        }
+        const float inv = 1.f / L;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const __nv_bfloat162 v = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
+          w[k >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+        }
+        const int64_t orow = (int64_t)row * TH + h;
+        *reinterpret_cast<uint4 *>(a.out + orow * TD + dh * DHALF + lane * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (a.lse && dh == 0 && lane == 0) a.lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
+      }
     }
+    // this CTA's shared memory stays valid until every peer has finished reading it
+    __syncthreads();
+    if (tid == 0)
+      for (uint32_t r = 0; r < S; ++r) peer_arrive(peer_addr(tc::smem_u32(&bars[BAR_MDONE]), r));
+    if (tid == 0) wait_cluster_bar(&bars[BAR_MDONE], a.status);
+    __syncthreads();
   }
-  const float inv = 1.f / L;
-  uint32_t w[8];
-#pragma unroll
-  for (int k = 0; k < 16; k += 2) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
-    w[k >> 1] = *reinterpret_cast<const uint32_t *>(&v);
-  }
-  uint4 *dst = reinterpret_cast<uint4 *>(out + ((int64_t)row * TH + h) * TD + lane * 16);
-  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  if (lse && lane == 0) lse[(int64_t)row * TH + h] = (M + log2f(L)) * 0.6931471805599453f;
+  if (warp == 8) tc::tmem_dealloc(tbase, TMEM_COLS);
 }
 
 }  // namespace
 
-// Splits per row so that rows * splits * 2 CTAs fill about one wave.
+// Item splits per (row, half): a power of two <= 8 (one thread-block cluster)
+// so that rows * 2 * splits CTAs fill about one wave of the SMs.
 static void tc_plan(const csa_dims *d, bool dense, int *splits, int *cps) {
   const int64_t rows = (int64_t)d->B * d->Tq;
   const int64_t max_items = (dense ? (int64_t)d->n_entries : (int64_t)d->K) + d->W;
   const int nch = (int)((max_items + CH - 1) / CH);
-  int s = (int)(148 / (2 * (rows > 0 ? rows : 1)));
-  if (s < 1) s = 1;
-  if (s > nch) s = nch;
+  const int64_t per = 148 / (2 * (rows > 0 ? rows : 1));
+  int s = 1;
+  while (s < 8 && 2 * s <= per && 2 * s <= nch) s *= 2;
   *cps = (nch + s - 1) / s;
-  *splits = (nch + *cps - 1) / *cps;
+  *splits = s;
 }
 
 bool attend_tc_supported(const csa_dims *d) { return d->H == TH && d->D == TD; }
 
-size_t attend_tc_workspace(const csa_dims *d, bool dense) {
-  int splits, cps;
-  tc_plan(d, dense, &splits, &cps);
-  if (splits == 1) return 0;
-  const int64_t rows = (int64_t)d->B * d->Tq;
-  return (size_t)(rows * splits * TH * (TD * 4 + 8)) + 256;
-}
+size_t attend_tc_workspace(const csa_dims *, bool) { return 0; }
 
 int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
                      const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
-                     const csa_dims *d, uint16_t *out, float *lse, void *workspace,
+                     const csa_dims *d, uint16_t *out, float *lse, void *,
                      cudaStream_t stream) {
   const bool dense = idx == nullptr;
   int splits, cps;
@@ -499,21 +601,26 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
   a.splits = splits; a.cps = cps;
   a.out = reinterpret_cast<__nv_bfloat16 *>(out);
   a.lse = lse;
-  a.ws_o = splits > 1 ? static_cast<float *>(workspace) : nullptr;
-  a.ws_ml = splits > 1 ? reinterpret_cast<float2 *>(static_cast<char *>(workspace) + (size_t)(rows * splits * TH * TD * 4)) : nullptr;
   a.status = status_word_device_ptr();
   if (int rc = set_smem_once((const void *)attend_tc_kernel, (int)SMEM_BYTES, "attend_tc_kernel")) return rc;
-  const int64_t grid = rows * splits * 2;
+  const int64_t grid = rows * 2 * splits;
   if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "attend: too many rows");
-  attend_tc_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, stream>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, a);
   count_launches(1);
-  if (int rc = check_launch("attend_tc_kernel")) return rc;
-  if (splits > 1) {
-    attend_merge_kernel<<<dim3((unsigned)rows, TH / 8), 256, 0, stream>>>(a.ws_o, a.ws_ml, splits, a.out, lse);
-    count_launches(1);
-    return check_launch("attend_merge_kernel");
-  }
-  return CSA_OK;
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attend_tc_kernel launch: %s", cudaGetErrorString(e));
+  return check_launch("attend_tc_kernel");
 }
 
 }  // namespace csa

@@ -21,6 +21,8 @@
 // radix select (12 bits per digit) over a shared-memory histogram, ties at
 // the threshold are resolved by index, and the K survivors are sorted with a
 // bitonic network.
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -392,8 +394,24 @@ __device__ void find_bin(const uint32_t *hist, uint32_t need, uint32_t *warp_tot
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int hi_bin = kBins - 1 - BPT * tid;
   uint32_t c[BPT], local = 0;
+  if (((uintptr_t)hist & 15u) == 0) {
+    // this thread's BPT bins are contiguous and 16-byte aligned: vector loads
+    // (scalar loads at a stride of BPT words would conflict on the banks)
+    const uint4 *h4 = reinterpret_cast<const uint4 *>(hist + hi_bin - (BPT - 1));
 #pragma unroll
-  for (int k = 0; k < BPT; ++k) { c[k] = hist[hi_bin - k]; local += c[k]; }
+    for (int k4 = 0; k4 < BPT / 4; ++k4) {
+      const uint4 v = h4[k4];
+      c[BPT - 1 - 4 * k4] = v.x;
+      c[BPT - 2 - 4 * k4] = v.y;
+      c[BPT - 3 - 4 * k4] = v.z;
+      c[BPT - 4 - 4 * k4] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) c[k] = hist[hi_bin - k];
+  }
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) local += c[k];
   uint32_t v = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -963,6 +981,516 @@ int launch_tc(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_
 }
 
 // ---------------------------------------------------------------------------
+// fused decode path: one cooperative launch, one CTA per SM, per_row CTAs per
+// query row, each owning a contiguous range of <= 8192 visible entries.
+//   scan     keys stream through a 4-stage ring of TMA tensor loads (32-byte
+//            swizzle, the layout the MMA reads); per 1024-key batch eight
+//            kind::mxf4 MMAs give exact q.k sums into one of two TMEM
+//            buffers, so the MMAs of batch b overlap the epilogue of b - 1;
+//            the integer scores stay in shared memory and are counted in a
+//            4096-bin histogram of score >> 8, which the CTA then adds into
+//            the row's global histogram.
+//   barrier  (bounded grid barrier)
+//   collect  every CTA finds the row's threshold bin b* and appends its keys
+//            of bin >= b* to the row's candidate list.  If b* holds so many
+//            keys that the list would overflow (heavy ties), the row is
+//            refined instead: a 256-bin histogram of the low score byte inside
+//            b* fixes the exact threshold score t*; keys above t* are taken,
+//            and the ties at t* in index order, each CTA taking its share after
+//            the tie counts of the CTAs before it (two more barriers, entered
+//            by the whole grid when any row needs them).
+//   rank     the candidates are unique 64-bit keys (score, ~index); each is
+//            ranked by counting the larger ones, spread over the row's CTAs,
+//            and written at its rank when that is below K.
+// ---------------------------------------------------------------------------
+constexpr int kFdThreads = 256;
+constexpr int kFdStages = 4;
+constexpr int kFdLocalCap = 8192;
+constexpr uint32_t kFdOffScores = kFdStages * kBatchBytes;            // u32 [8192]
+constexpr uint32_t kFdOffHist = kFdOffScores + kFdLocalCap * 4;       // u32 [4096]
+constexpr uint32_t kFdOffQ = kFdOffHist + kBins * 4;                  // 8 rows x 32 B
+constexpr uint32_t kFdOffBar = kFdOffQ + 256;
+constexpr uint32_t kFdOffMisc = kFdOffBar + 64;
+constexpr uint32_t kFdSmem = kFdOffMisc + 256;
+constexpr uint32_t kFdTmemCols = 256;                                 // 2 x 64 accumulator + scale columns
+constexpr uint32_t kFdColSFA = 128, kFdColSFB = 132;
+
+struct FdWs {
+  uint64_t *cand;     // [rows][kCandCap]
+  uint32_t *hist;     // [rows][4096]     (zeroed per call from here on)
+  uint32_t *hist2;    // [rows][256]
+  uint32_t *ccount;   // [rows]
+  uint32_t *tiecnt;   // [rows * per_row]
+  uint32_t *sync;     // grid barrier counter
+  uint32_t *flag;     // some row needs the refinement
+};
+
+struct FdMisc {
+  uint32_t tmem;
+  int abort;
+  SelShared sel;
+  uint32_t cnt[8];
+  uint32_t tstar, take, base;
+};
+
+// Bounded grid barrier number k (1, 2, ...) over G CTAs of a cooperative
+// launch: arrive, then wait until all G arrived.  A CTA whose wait gave up
+// raises STATUS_TIMEOUT and stops waiting at later barriers (it still arrives).
+__device__ __forceinline__ void fd_grid_barrier(uint32_t *ctr, uint32_t k, uint32_t G, FdMisc *misc,
+                                                unsigned *status) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // release: the CTA's writes (ordered before by the CTA barrier) become
+    // visible before the arrival; acquire on the loads that see all arrivals
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+    if (!misc->abort) {
+      const uint64_t t0 = gtimer();
+      uint32_t v, n = 0;
+      for (;;) {
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= k * G) break;
+        if ((++n & 63u) == 0 && gtimer() - t0 > kScanWaitNs) {
+          misc->abort = 1;
+          raise_status(status, STATUS_TIMEOUT);
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Warp-aggregated append of `key` (when take) to a global list with counter.
+__device__ __forceinline__ void fd_append(bool take, uint64_t key, uint32_t *count, uint64_t *list, uint32_t cap) {
+  const int lane = threadIdx.x & 31;
+  const unsigned msk = __ballot_sync(0xffffffffu, take);
+  if (!msk) return;
+  const int leader = __ffs(msk) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(count, (uint32_t)__popc(msk));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (take) {
+    const uint32_t pos = base + __popc(msk & ((1u << lane) - 1u));
+    if (pos < cap) list[pos] = key;
+  }
+}
+
+// Exclusive prefix of v over the CTA (kFdThreads threads) and the total.
+__device__ __forceinline__ uint32_t fd_block_scan(uint32_t v, uint32_t *warp_tot, uint32_t *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  uint32_t before = 0, tot = 0;
+#pragma unroll
+  for (int k = 0; k < kFdThreads / 32; ++k) {
+    const uint32_t t = warp_tot[k];
+    before += (k < warp) ? t : 0u;
+    tot += t;
+  }
+  *total = tot;
+  return before + x - v;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kFdThreads, 1)
+index_decode_kernel(const __grid_constant__ CUtensorMap kmap, const uint8_t *__restrict__ qI,
+                    const float *__restrict__ w, const int32_t *__restrict__ q_pos, int Tq, int m, int n_entries,
+                    int64_t entry_cap, int K, int per_row, FdWs ws, int32_t *__restrict__ idx_out,
+                    float *__restrict__ score_out, unsigned *status) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char *kbuf = smem;
+  uint32_t *sc = reinterpret_cast<uint32_t *>(smem + kFdOffScores);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem + kFdOffHist);
+  unsigned char *qbuf = smem + kFdOffQ;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kFdOffBar);
+  FdMisc *misc = reinterpret_cast<FdMisc *>(smem + kFdOffMisc);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t G = gridDim.x;
+  const int row = blockIdx.x / per_row, part = blockIdx.x - row * per_row;
+  const int b = row / Tq;
+  const int64_t t = q_pos[row];
+  if (t < 0 && tid == 0 && part == 0) raise_status(status, STATUS_BAD_POSITION);
+  const int nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
+  const int slice = (nvis + per_row - 1) / per_row;
+  const int s0 = min(part * slice, nvis), s1 = min(s0 + slice, nvis);
+  const int n = s1 - s0;
+  const int nb = (n + kBatchKeys - 1) / kBatchKeys;
+  const int ybase = (int)((int64_t)b * entry_cap + s0);    // row of the key tensor (< 2^31)
+  uint64_t *full = bar;                                    // [kFdStages] key batch landed
+  uint64_t *mdone = bar + kFdStages;                       // [2] accumulator buffer complete
+  // batch bb: keys [bb * 1024, +1024) of the range, as 256-row TMA boxes
+  // (boxes wholly past the range are skipped; rows past it inside a box are
+  // loaded and masked)
+  auto issue = [&](int bb) {
+    const int slot = bb % kFdStages;
+    const int boxes = min(4, (n - bb * kBatchKeys + 255) >> 8);
+    tc::mbar_arrive_expect_tx(&full[slot], (uint32_t)boxes * 8192u);
+    for (int i = 0; i < boxes; ++i)
+      tc::tma_load_2d(kbuf + slot * kBatchBytes + i * 8192, &kmap, 0, ybase + bb * kBatchKeys + i * 256,
+                      &full[slot]);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kFdStages + 2; ++i) tc::mbar_init(&bar[i], 1);
+    misc->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int bb = 0; bb < min(kFdStages, nb); ++bb) issue(bb);
+  }
+  if (warp == 0) tc::tmem_alloc(&misc->tmem, kFdTmemCols);
+  for (int i = tid; i < kBins; i += kFdThreads) hist[i] = 0;
+  if (tid < 16) {
+    const int r = tid & 7, c = tid >> 3;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < HI) v = *reinterpret_cast<const uint4 *>(qI + ((int64_t)row * HI + r) * 32 + c * 16);
+    *reinterpret_cast<uint4 *>(qbuf + c * 128 + r * 16) = v;
+  }
+  int w16[HI];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) {
+    const float f = w[(int64_t)row * HI + h] * 16.f;
+    w16[h] = __float2int_rn(f);
+    if (tid == 0 && part == 0 && ((float)w16[h] != f || w16[h] < 0 || w16[h] > 16))
+      raise_status(status, STATUS_BAD_WEIGHT);
+  }
+  tc::fence_proxy_async_smem();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = misc->tmem;
+  if (warp < 4) {     // block scales = 2^0 (UE8M0 127) in every byte the MMA may read
+    const uint32_t ones[4] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kFdColSFA, ones);
+    tc::tmem_st4(tbase + ((uint32_t)(warp * 32) << 16) + kFdColSFB, ones);
+    tc::tmem_wait_st();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+
+  // bounded wait on an mbarrier phase; gives up (and marks the CTA) after 2 s
+  auto bwait = [&](uint64_t *bb_, uint32_t par) -> bool {
+    if (*(volatile int *)&misc->abort) return false;
+    if (tc::mbar_try_wait(bb_, par)) return true;
+    const uint64_t t0 = gtimer();
+    uint32_t it = 0;
+    while (!tc::mbar_try_wait(bb_, par)) {
+      if ((++it & 255u) == 0 && (*(volatile int *)&misc->abort || gtimer() - t0 > kScanWaitNs)) {
+        if (!*(volatile int *)&misc->abort) raise_status(status, STATUS_TIMEOUT);
+        *(volatile int *)&misc->abort = 1;
+        return false;
+      }
+    }
+    return true;
+  };
+
+  // ---- scan
+  const uint32_t idesc = tc::idesc_mxf4(128, 8);
+  const uint64_t bd = tc::smem_desc(tc::smem_u32(qbuf), 128, 256);
+  for (int bb = 0; bb <= nb; ++bb) {
+    if (bb < nb && tid == 0) {
+      const int slot = bb % kFdStages;
+      if (bwait(&full[slot], (uint32_t)(bb / kFdStages) & 1u)) {
+        tc::fence_after_sync();
+        const uint32_t buf = tc::smem_u32(kbuf + slot * kBatchBytes);
+        const uint32_t acc = tbase + (uint32_t)(bb & 1) * 64;
+#pragma unroll
+        for (int i = 0; i < kBatchTiles; ++i)
+          tc::mma_mxf4_ss(acc + i * 8, tc::smem_desc_sw32(buf + i * 4096), bd, idesc, tbase + kFdColSFA,
+                          tbase + kFdColSFB, 0);
+      }
+      tc::mma_commit(&mdone[bb & 1]);
+    }
+    if (bb > 0) {
+      const int pb = bb - 1;
+      const bool ok = bwait(&mdone[pb & 1], (uint32_t)(pb >> 1) & 1u);
+      tc::fence_after_sync();
+      // the key slot of batch pb is free again
+      if (tid == 0 && pb + kFdStages < nb) issue(pb + kFdStages);
+      const int q = warp & 3;
+      uint32_t acc[4][4];
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        acc[i4][0] = acc[i4][1] = acc[i4][2] = acc[i4][3] = 0u;
+        if (ok) tc::tmem_ld4(tbase + ((uint32_t)(q * 32) << 16) + (uint32_t)(pb & 1) * 64 + ((warp >> 2) * 4 + i4) * 8,
+                             acc[i4]);
+      }
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int tile = (warp >> 2) * 4 + i4;
+        const int j = pb * kBatchKeys + tile * kTileKeys + q * 32 + lane;   // local index
+        const bool valid = j < n;
+        uint32_t s = 0;
+#pragma unroll
+        for (int h = 0; h < HI; ++h)
+          s += (uint32_t)(w16[h] * max(0, __float2int_rn(4.f * __uint_as_float(acc[i4][h]))));
+        if (valid) {
+          sc[j] = s;
+          atomicAdd(&hist[s >> 8], 1u);
+        }
+      }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+  }
+  // add the CTA's histogram into the row's (the scores occupy few bins)
+  uint32_t *ghist = ws.hist + (int64_t)row * kBins;
+  for (int i = tid; i < kBins; i += kFdThreads) {
+    const uint32_t c = hist[i];
+    if (c) atomicAdd(&ghist[i], c);
+  }
+  fd_grid_barrier(ws.sync, 1, G, misc, status);
+
+  // ---- collect
+  uint32_t bstar = 0, above = 0, C = (uint32_t)nvis;
+  if (nvis > K) {
+    const uint4 *G4 = reinterpret_cast<const uint4 *>(ghist);
+    for (int i = tid; i < kBins / 4; i += kFdThreads) reinterpret_cast<uint4 *>(hist)[i] = __ldcg(G4 + i);
+    __syncthreads();
+    find_bin<kFdThreads>(hist, (uint32_t)K, misc->sel.warp_tot, &misc->sel.bin, &misc->sel.above);
+    bstar = (uint32_t)misc->sel.bin;
+    above = misc->sel.above;
+    C = above + hist[bstar];
+  }
+  const bool refine = C > (uint32_t)kCandCap;
+  uint64_t *cand = ws.cand + (int64_t)row * kCandCap;
+  uint32_t *ccount = ws.ccount + row;
+  if (!refine) {
+    // count, reserve the CTA's block of the list with one atomic, then write
+    uint32_t mine = 0;
+    for (int j = tid; j < n; j += kFdThreads) mine += (sc[j] >> 8) >= bstar ? 1u : 0u;
+    uint32_t total;
+    uint32_t pos = fd_block_scan(mine, misc->cnt, &total);
+    if (tid == 0) misc->base = total ? atomicAdd(ccount, total) : 0u;
+    __syncthreads();
+    pos += misc->base;
+    for (int j = tid; j < n; j += kFdThreads) {
+      const uint32_t s = sc[j];
+      if ((s >> 8) >= bstar) {
+        if (pos < (uint32_t)kCandCap) cand[pos] = make_key(s, (uint32_t)(s0 + j));
+        ++pos;
+      }
+    }
+  } else {
+    if (tid == 0 && part == 0) atomicOr(ws.flag, 1u);
+    __syncthreads();
+    for (int i = tid; i < 256; i += kFdThreads) hist[i] = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += kFdThreads) {
+      const uint32_t s = sc[j];
+      if ((s >> 8) == bstar) atomicAdd(&hist[s & 255u], 1u);
+    }
+    __syncthreads();
+    for (int i = tid; i < 256; i += kFdThreads)
+      if (hist[i]) atomicAdd(&ws.hist2[row * 256 + i], hist[i]);
+  }
+  fd_grid_barrier(ws.sync, 2, G, misc, status);
+
+  if (*(volatile uint32_t *)ws.flag) {       // the same decision in every CTA
+    uint32_t tstar = 0, take_ties = 0;
+    if (refine) {
+      if (tid == 0) {
+        const uint32_t need = (uint32_t)K - above;
+        uint32_t run = 0;
+        int lo = 255;
+        for (; lo > 0; --lo) {
+          const uint32_t c = __ldcg(ws.hist2 + row * 256 + lo);
+          if (run + c >= need) break;
+          run += c;
+        }
+        misc->tstar = (bstar << 8) | (uint32_t)lo;
+        misc->take = need - run;   // ties at t* to take
+      }
+      __syncthreads();
+      tstar = misc->tstar;
+      take_ties = misc->take;
+      uint32_t myties = 0;
+      for (int j0 = 0; j0 < n; j0 += kFdThreads) {
+        const int j = j0 + tid;
+        const uint32_t s = j < n ? sc[j] : 0u;
+        fd_append(j < n && s > tstar, make_key(s, (uint32_t)(s0 + j)), ccount, cand, kCandCap);
+        myties += (j < n && s == tstar) ? 1u : 0u;
+      }
+      myties = __reduce_add_sync(0xffffffffu, myties);
+      if (lane == 0) misc->cnt[warp] = myties;
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t tot = 0;
+        for (int k = 0; k < kFdThreads / 32; ++k) tot += misc->cnt[k];
+        ws.tiecnt[blockIdx.x] = tot;
+      }
+      __syncthreads();
+    }
+    fd_grid_barrier(ws.sync, 3, G, misc, status);
+    if (refine) {
+      // ties before this CTA's range, then this CTA's first (take - before) ties in index order
+      uint32_t before = 0;
+      for (int p = 0; p < part; ++p) before += __ldcg(ws.tiecnt + row * per_row + p);
+      const uint32_t want = take_ties > before ? take_ties - before : 0u;
+      if (warp == 0 && want > 0) {
+        uint32_t got = 0;
+        for (int j0 = 0; j0 < n && got < want; j0 += 32) {
+          const int j = j0 + lane;
+          const bool tie = j < n && sc[j] == tstar;
+          const unsigned msk = __ballot_sync(0xffffffffu, tie);
+          const uint32_t r = got + __popc(msk & ((1u << lane) - 1u));
+          fd_append(tie && r < want, make_key(tstar, (uint32_t)(s0 + j)), ccount, cand, kCandCap);
+          got += __popc(msk);
+        }
+      }
+    }
+    fd_grid_barrier(ws.sync, 4, G, misc, status);
+  }
+
+  // ---- rank
+  const int cnt = min(K, nvis);
+  int32_t *oi = idx_out + (int64_t)row * K;
+  float *os = score_out ? score_out + (int64_t)row * K : nullptr;
+  const uint32_t nc = min(__ldcg(ccount), (uint32_t)kCandCap);
+  uint64_t *ck = reinterpret_cast<uint64_t *>(kbuf);   // the key ring is idle now
+  for (uint32_t i = tid; i < nc; i += kFdThreads) ck[i] = __ldcg(cand + i);
+  __syncthreads();
+  for (uint32_t i = (uint32_t)(part + per_row * warp); i < nc; i += (uint32_t)(per_row * (kFdThreads / 32))) {
+    const uint64_t key = ck[i];
+    uint32_t r = 0;
+    for (uint32_t j = lane; j < nc; j += 32) r += ck[j] > key ? 1u : 0u;
+    r = __reduce_add_sync(0xffffffffu, r);
+    if (lane == 0 && r < (uint32_t)cnt) {
+      oi[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu));
+      if (os) os[r] = (float)(uint32_t)(key >> 32) * (1.f / 64.f);
+    }
+  }
+  if (part == 0) {
+    for (int j = cnt + tid; j < K; j += kFdThreads) {
+      oi[j] = -1;
+      if (os) os[j] = 0.f;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tbase, kFdTmemCols);
+}
+
+int fd_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cache[dev]) {
+    int sms = 0, occ = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    if (set_smem_once((const void *)index_decode_kernel<4>, (int)kFdSmem, "index_decode_kernel")) return 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, index_decode_kernel<4>, kFdThreads, kFdSmem) !=
+            cudaSuccess || occ < 1)
+      return 0;
+    cache[dev] = sms;   // one CTA per SM
+  }
+  return cache[dev];
+}
+
+// Fused decode plan: per_row CTAs per row, all co-resident (one per SM).
+bool fd_plan(const csa_dims *d, int *per_row) {
+  const int rows = d->B * d->Tq;
+  if (d->dI != 64 || d->HI > 4 || d->HI < 1 || rows < 1 || d->K > kCandCap || d->n_entries < 1) return false;
+  const int sms = fd_sms();
+  if (sms < 1 || rows > sms) return false;
+  const int pr = sms / rows;
+  if ((d->n_entries + pr - 1) / pr > kFdLocalCap) return false;
+  *per_row = pr;
+  return true;
+}
+
+size_t fd_workspace(const csa_dims *d, int per_row, FdWs *ws, void *base, size_t *zero_off) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
+  const size_t o_cand = take((size_t)(rows * kCandCap * 8));
+  const size_t o_hist = take((size_t)(rows * kBins * 4));
+  const size_t o_hist2 = take((size_t)(rows * 256 * 4));
+  const size_t o_cnt = take((size_t)(rows * 4));
+  const size_t o_tie = take((size_t)(rows * per_row * 4));
+  const size_t o_sync = take(4);
+  const size_t o_flag = take(4);
+  if (zero_off) *zero_off = o_hist;
+  if (ws && base) {
+    char *p = static_cast<char *>(base);
+    ws->cand = reinterpret_cast<uint64_t *>(p + o_cand);
+    ws->hist = reinterpret_cast<uint32_t *>(p + o_hist);
+    ws->hist2 = reinterpret_cast<uint32_t *>(p + o_hist2);
+    ws->ccount = reinterpret_cast<uint32_t *>(p + o_cnt);
+    ws->tiecnt = reinterpret_cast<uint32_t *>(p + o_tie);
+    ws->sync = reinterpret_cast<uint32_t *>(p + o_sync);
+    ws->flag = reinterpret_cast<uint32_t *>(p + o_flag);
+  }
+  return off;
+}
+
+// Tensor map over the indexer keys viewed as [B * entry_cap rows][32 bytes],
+// 256-row boxes, 32-byte swizzle (the layout the MMA descriptor reads).
+bool fd_key_map(const uint8_t *kI, const csa_dims *d, CUtensorMap *map) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const int64_t rows = (int64_t)d->B * d->entry_cap;
+  if (((uintptr_t)kI & 15u) != 0 || rows < 1 || rows >= (1ll << 31)) return false;
+  const cuuint64_t dims[2] = {32, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {32};
+  const cuuint32_t box[2] = {32, 256};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(kI), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_fd(const CUtensorMap &kmap, const uint8_t *qI, const float *w, const int32_t *q_pos, const csa_dims *d,
+              int per_row, int32_t *idx_out, float *score_out, void *workspace, cudaStream_t stream) {
+  FdWs ws;
+  size_t zoff = 0;
+  const size_t total = fd_workspace(d, per_row, &ws, workspace, &zoff);
+  if (cudaMemsetAsync(static_cast<char *>(workspace) + zoff, 0, total - zoff, stream) != cudaSuccess)
+    return check_launch("cudaMemsetAsync");
+  const int rows = d->B * d->Tq;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(rows * per_row));
+  cfg.blockDim = dim3(kFdThreads);
+  cfg.dynamicSmemBytes = kFdSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  unsigned *st = status_word_device_ptr();
+  cudaError_t e;
+  switch (d->HI) {
+    case 1: if (set_smem_once((const void *)index_decode_kernel<1>, (int)kFdSmem, "index_decode_kernel")) return CSA_ERR_CUDA;
+            e = cudaLaunchKernelEx(&cfg, index_decode_kernel<1>, kmap, qI, w, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, per_row, ws, idx_out, score_out, st); break;
+    case 2: if (set_smem_once((const void *)index_decode_kernel<2>, (int)kFdSmem, "index_decode_kernel")) return CSA_ERR_CUDA;
+            e = cudaLaunchKernelEx(&cfg, index_decode_kernel<2>, kmap, qI, w, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, per_row, ws, idx_out, score_out, st); break;
+    case 3: if (set_smem_once((const void *)index_decode_kernel<3>, (int)kFdSmem, "index_decode_kernel")) return CSA_ERR_CUDA;
+            e = cudaLaunchKernelEx(&cfg, index_decode_kernel<3>, kmap, qI, w, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, per_row, ws, idx_out, score_out, st); break;
+    default: e = cudaLaunchKernelEx(&cfg, index_decode_kernel<4>, kmap, qI, w, q_pos, d->Tq, d->m, d->n_entries, d->entry_cap, d->K, per_row, ws, idx_out, score_out, st); break;
+  }
+  count_launches(1);
+  if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "index_decode_kernel launch: %s", cudaGetErrorString(e));
+  return check_launch("index_decode_kernel");
+}
+
+// ---------------------------------------------------------------------------
 // tensor-core prefill path: one CTA per 128 query rows (one TMEM lane per
 // query), streaming 16-entry key tiles.  Per tile and head one kind::mxf4 MMA
 // (M = 128 queries, N = 16 entries, K = 64) gives exact q.k sums; each
@@ -1282,7 +1810,13 @@ int launch_prefill_tc(const uint8_t *qI, const float *w, const uint8_t *kI, cons
 }  // namespace
 
 size_t index_topk_workspace(const csa_dims *d) {
-  int splits, slice;
+  int splits, slice, per_row;
+  if (fd_plan(d, &per_row)) {
+    // the launch falls back to the two-kernel path when the keys cannot be mapped
+    const size_t a = fd_workspace(d, per_row, nullptr, nullptr, nullptr);
+    const size_t b = tc_plan(d, &splits, &slice) ? tc_workspace(d, nullptr, nullptr) : 0;
+    return a > b ? a : b;
+  }
   if (tc_plan(d, &splits, &slice)) return tc_workspace(d, nullptr, nullptr);
   if (prefill_tc_plan(d)) return (size_t)((int64_t)d->B * d->Tq * d->K * 4);
   if (split_plan(d, &splits, &slice)) return (size_t)((int64_t)d->B * d->Tq * splits * d->K * 8);
@@ -1296,7 +1830,12 @@ int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, cons
   const int rows = d->B * d->Tq;
   if (rows == 0) return CSA_OK;
   if (d->K > kMaxK) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: K > %d", kMaxK);
-  int splits, slice;
+  int splits, slice, per_row;
+  if (fd_plan(d, &per_row)) {
+    CUtensorMap kmap;
+    if (fd_key_map(kI, d, &kmap))
+      return launch_fd(kmap, qI, w, q_pos, d, per_row, idx_out, score_out, workspace, stream);
+  }
   if (tc_plan(d, &splits, &slice))
     return launch_tc(qI, w, kI, q_pos, d, splits, slice, idx_out, score_out, workspace, stream);
   if (prefill_tc_plan(d)) return launch_prefill_tc(qI, w, kI, q_pos, d, idx_out, score_out, workspace, stream);
