@@ -15,11 +15,14 @@
 // across the CTA's chunks of 32 items.  Both halves of a row compute the same
 // S (each needs the full 512-wide dot products) and keep bit-identical softmax
 // state, so their halves combine without exchange.  The item splits of one
-// (row, half) (1, 2, 4 or 8) form a thread-block cluster: each CTA parks its
-// unnormalised partial O and per-head (max, sum) in its own shared memory and
-// the CTAs merge them through distributed shared memory, each producing the
-// final rows of 128 / splits heads:
+// (row, half) (1, 2, 4 or 8) form a thread-block cluster: each CTA writes its
+// unnormalised partial O and per-head (max, sum) to the workspace (L2), one
+// hardware cluster barrier orders them, and CTA c then combines the final
+// rows of heads [c * 128 / S, +128 / S):
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
+// Q arrives by 32 TMA boxes of 128 heads x 16 d (32-byte swizzle, the layout
+// the MMA reads); the CTA's gathered rows are prefetched into L2 right after
+// the selection is compacted.
 //
 // Roles (288 threads):
 //   warps 0-3  gather 32 items per chunk, convert E4M3 codes exactly to bf16
@@ -66,7 +69,7 @@ constexpr uint32_t TCOL_S = 256;      // 2 x 32 columns
 constexpr uint32_t TMEM_COLS = 512;
 
 enum { BAR_KV_FULL = 0, BAR_KV_FREE = 2, BAR_S_FULL = 4, BAR_P_FULL = 6, BAR_PV_DONE = 8, BAR_FIN = 9,
-       BAR_MREADY = 10, BAR_MDONE = 11, BAR_Q = 12 };
+       BAR_Q = 10 };
 
 struct Misc {
   uint32_t tmem_base;
@@ -99,71 +102,18 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Misc *m
   return true;
 }
 
-// ---- cluster helpers (distributed shared memory)
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void peer_arrive(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
-__device__ __forceinline__ bool try_wait_cluster(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(tc::smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait (acquire at cluster scope) for the first phase of `bar`.
-__device__ __forceinline__ bool wait_cluster_bar(uint64_t *bar, unsigned *status) {
-  const uint64_t t0 = globaltimer();
-  uint32_t n = 0;
-  while (!try_wait_cluster(bar, 0)) {
-    if ((++n & 255u) == 0 && globaltimer() - t0 > kWaitNs) {
-      raise_status(status, STATUS_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ float4 ld_peer_f4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float2 ld_peer_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-
-// Partial O in shared memory for the cluster merge: fp32 [128 heads][256 d]
-// over the Q region, 16-byte chunk c of head h at chunk c ^ (h & 7) (the
-// eight heads of a store phase hit distinct banks); (max, sum) per head in
-// the selection region.
-__device__ __forceinline__ uint32_t po_off(int h, int c) { return (uint32_t)h * 1024 + ((c ^ (h & 7)) << 4); }
 
 // Byte offsets in the core-matrix layouts.  g counts 16-byte groups along
 // the contraction-side dimension of each tile (8 bf16).  Every tile keeps
 // the 8-row-group stride at 128 B and the other stride at most 2 KiB, so all
 // descriptor strides stay small.
-//   Q  [128 heads][512 d]:  g = d/8,     g-stride 2048 B, head-group stride 128 B
+//   Q  [128 heads][512 d]:  not core matrices: 32 TMA boxes [128 heads][16 d]
+//                           of 4 KiB with 32-byte swizzle, box k at k * 4096
 //   KV [32 items][512 d]:   g = d/8,     g-stride 512 B,  item-group stride 128 B
 //   P  [128 heads][32 items]: g = item/8, g-stride 2048 B, head-group stride 128 B
-__device__ __forceinline__ uint32_t q_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
 __device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 512 + (i >> 3) * 128 + (i & 7) * 16; }
 __device__ __forceinline__ uint32_t p_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
 
@@ -198,10 +148,13 @@ struct Args {
   int splits, cps;          // splits per row, chunks per split
   __nv_bfloat16 *out;
   float *lse;
+  float *ws_o;              // [rows * 2][splits][8 blocks][128][32] partial outputs (splits > 1)
+  float2 *ws_ml;            // [rows * 2][splits][128] (max, sum) in log2 units
   unsigned *status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                                                                const Args a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   Misc *misc = reinterpret_cast<Misc *>(smem + OFF_MISC);
@@ -228,77 +181,89 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
     misc->abort = 0;
     for (int i = 0; i < 10; ++i) tc::mbar_init(&bars[i], (i == BAR_KV_FULL || i == BAR_KV_FULL + 1) ? 128
                                                        : (i == BAR_P_FULL || i == BAR_P_FULL + 1) ? 128 : 1);
-    tc::mbar_init(&bars[BAR_MREADY], (uint32_t)a.splits);
-    tc::mbar_init(&bars[BAR_MDONE], (uint32_t)a.splits);
-    tc::mbar_init(&bars[BAR_Q], 128);
+    tc::mbar_init(&bars[BAR_Q], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (a.splits > 1) {
-    // every CTA of the cluster has initialised its barriers before any remote arrival
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-  }
-  if (warp == 8) tc::tmem_alloc(&misc->tmem_base, TMEM_COLS);
-
-  // ordered compaction of the valid selected entries
-  int nsel;
-  if (a.idx) {
+  __syncthreads();
+  if (warp == 8) {
+    tc::tmem_alloc(&misc->tmem_base, TMEM_COLS);
+  } else if (a.idx) {
+    // ordered compaction of the valid selected entries (warps 0-7)
     const int32_t *irow = a.idx + (int64_t)row * a.K;
     int base = 0;
-    for (int j0 = 0; j0 < a.K; j0 += kThreads) {
+    for (int j0 = 0; j0 < a.K; j0 += 256) {
       const int j = j0 + tid;
       int e = (j < a.K) ? irow[j] : -1;
       if (e >= a.n_entries || e < -1) { raise_status(a.status, STATUS_BAD_INDEX); e = -1; }
       const bool f = e >= 0;
       const unsigned bal = __ballot_sync(0xffffffffu, f);
       if (lane == 0) misc->wcount[warp] = __popc(bal);
-      __syncthreads();
+      asm volatile("bar.sync 2, 256;" ::: "memory");
       int before = 0, tot = 0;
-      for (int k = 0; k < kThreads / 32; ++k) { if (k < warp) before += misc->wcount[k]; tot += misc->wcount[k]; }
+      for (int k = 0; k < 8; ++k) { if (k < warp) before += misc->wcount[k]; tot += misc->wcount[k]; }
       if (f) sel[base + before + __popc(bal & ((1u << lane) - 1u))] = e;
       base += tot;
-      __syncthreads();
+      asm volatile("bar.sync 2, 256;" ::: "memory");
     }
-    nsel = base;
-  } else {
-    nsel = nvis;
+    if (tid == 0) misc->nsel = base;
   }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const int nsel = a.idx ? misc->nsel : nvis;
   const int n_items = nsel + nwin;
   const int nch = (n_items + CH - 1) / CH;
   const int c_begin = split * a.cps;
   const int c_end = min(c_begin + a.cps, nch);
   const int nloc = max(0, c_end - c_begin);
-
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
   const uint32_t tbase = misc->tmem_base;
   const uint32_t sbase = tc::smem_u32(smem);
+  if (warp == 8) {
+    // Q (32 boxes of 128 heads x 16 d, 32-byte swizzle: box k is the A
+    // operand of the k-th K step) while the loaders gather the first chunks
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(&bars[BAR_Q], TH * TD * 2);
+      for (int k = 0; k < TD / 16; ++k) tc::tma_load_2d(smem + OFF_Q + k * 4096, &qmap, 16 * k, row * TH, &bars[BAR_Q]);
+    }
+    // pull this CTA's gathered rows into L2 ahead of the loaders
+    const int u1 = min(c_end * CH, n_items);
+    for (int u = c_begin * CH + lane; u < u1; u += 32) {
+      const uint8_t *src;
+      if (u < nsel) src = a.codes + ((int64_t)b * a.entry_cap + (a.idx ? sel[u] : u)) * TD;
+      else src = a.wcodes + ((int64_t)b * a.win_cap + ((p0 + (u - nsel)) % a.win_cap)) * TD;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(TD) : "memory");
+    }
+  }
 
   if (warp < 4) {
     // ------------------------------------------------------------ loaders
     const int i8 = lane & 7, pq = lane >> 3;
     for (int lc = 0; lc < nloc; ++lc) {
       const int buf = lc & 1;
-      if (lc >= 2 && !wait_bar(&bars[BAR_KV_FREE + buf], ((lc - 2) >> 1) & 1, misc, a.status)) break;
       const int item = warp * 8 + i8;
       const int u = (c_begin + lc) * CH + item;
-      const uint8_t *src = nullptr;
-      float sc = 0.f;
+      // Items past the list read a valid row (the first window token): their
+      // logits are masked and their P is zero, so the finite codes do not
+      // matter.  The loads are issued before waiting for the buffer.
+      const uint8_t *src;
+      const float *scp;
       if (u < nsel) {
         const int e = a.idx ? sel[u] : u;
         const int64_t ent = (int64_t)b * a.entry_cap + e;
         src = a.codes + ent * TD;
-        sc = a.scales[ent];
-      } else if (u < n_items) {
-        const int64_t p = p0 + (u - nsel);
+        scp = a.scales + ent;
+      } else {
+        const int64_t p = p0 + (u < n_items ? u - nsel : 0);
         const int64_t ent = (int64_t)b * a.win_cap + (p % a.win_cap);
         src = a.wcodes + ent * TD;
-        sc = a.wscales[ent];
+        scp = a.wscales + ent;
       }
       uint4 c[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        c[k] = src ? __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * k) : make_uint4(0, 0, 0, 0);
+      for (int k = 0; k < 8; ++k) c[k] = __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * k);
+      const float sc_raw = __ldg(scp);
+      if (lc >= 2 && !wait_bar(&bars[BAR_KV_FREE + buf], ((lc - 2) >> 1) & 1, misc, a.status)) break;
+      const float sc = u < n_items ? sc_raw : 0.f;
       unsigned char *kv = smem + OFF_KV + buf * KV_BYTES;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -314,30 +279,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    // Q -> shared memory (core-matrix layout) while the loaders gather the
-    // first chunks; lane pairs read 32 contiguous bytes of one head, a warp
-    // covers 16 heads; 8 loads in flight per thread
-    if (nloc > 0) {
-      const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * TH * TD);
-      const int t = tid - 128;
-#pragma unroll 1
-      for (int it0 = 0; it0 < (TH * TD / 8) / 128; it0 += 8) {
-        uint4 v[8];
-        int hh[8], gg[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          // idx bits: [0] g_lo, [1..4] h_lo, [5..6] h_hi, [7..12] g_hi
-          const int idx = (it0 + u) * 128 + t;
-          hh[u] = ((idx >> 5) & 3) * 16 + ((idx >> 1) & 15) + 64 * ((idx >> 7) & 1);
-          gg[u] = (idx >> 8) * 2 + (idx & 1);
-          v[u] = __ldg(qrow + hh[u] * (TD / 8) + gg[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) *reinterpret_cast<uint4 *>(smem + OFF_Q + q_off(hh[u], gg[u])) = v[u];
-      }
-      tc::fence_proxy_async_smem();
-    }
-    tc::mbar_arrive(&bars[BAR_Q]);
     const int quad = warp - 4;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -425,8 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
         if (a.lse && dh == 0) a.lse[orow] = (m_used + log2f(l)) * 0.6931471805599453f;
       }
     } else {
-      // park the partial (zeros when this split had no items) for the merge;
-      // the Q tile is no longer read once the last PV has completed
+      // partial rows (zeros when this split had no items) straight from TMEM
+      // to the workspace, laid out [32-column block][head][32] so that each
+      // thread writes whole 128-byte lines
+      const int64_t slot = (int64_t)pair * a.splits + split;
+      float *dstb = a.ws_o + slot * TH * DHALF;
 #pragma unroll 1
       for (int blk = 0; blk < DHALF / 32; ++blk) {
         uint32_t o[32];
@@ -437,16 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = 0u;
         }
+        uint4 *dst = reinterpret_cast<uint4 *>(dstb + ((int64_t)blk * TH + h) * 32);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          *reinterpret_cast<uint4 *>(smem + OFF_Q + po_off(h, blk * 8 + k)) =
-              make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        for (int k = 0; k < 8; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
       }
-      reinterpret_cast<float2 *>(smem + OFF_SEL)[h] = have ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
-      asm volatile("fence.acq_rel.cluster;" ::: "memory");   // visible to the peers' reads
+      a.ws_ml[slot * TH + h] = have ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
     }
   } else {
-    // ------------------------------------------------------------ MMA issuer  } else {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nloc > 0) {
       const uint32_t idesc_qk = tc::idesc_bf16_f32(128, CH, 0, 0);
@@ -456,8 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
         const uint32_t kvb = sbase + OFF_KV + buf * KV_BYTES;
 #pragma unroll 4
         for (int k = 0; k < TD / 16; ++k) {
-          // K-major A (Q) and B (items): LBO = step between d-groups, SBO = 8-row groups
-          const uint64_t ad = tc::smem_desc(sbase + OFF_Q + k * 4096, 2048, 128);
+          // A = Q, K-major with 32-byte swizzle (one TMA box per K step);
+          // B = items, K-major core matrices: LBO = step between d-groups, SBO = 8-row groups
+          const uint64_t ad = tc::smem_desc_sw32(sbase + OFF_Q + k * 4096);
           const uint64_t bd = tc::smem_desc(kvb + k * 1024, 512, 128);
           tc::mma_bf16_ss(tbase + TCOL_S + buf * CH, ad, bd, idesc_qk, k > 0);
         }
@@ -503,19 +445,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
   tc::fence_after_sync();
 
   if (a.splits > 1) {
-    // ---- cluster merge: heads [rank * 128 / S, +128 / S) of this (row, half)
-    const uint32_t S = (uint32_t)a.splits;
-    const uint32_t rank = cluster_rank();
-    if (tid == 0)
-      for (uint32_t r = 0; r < S; ++r) peer_arrive(peer_addr(tc::smem_u32(&bars[BAR_MREADY]), r));
-    const bool ready = wait_cluster_bar(&bars[BAR_MREADY], a.status);
-    if (ready && warp < 8) {
-      const int hper = TH / (int)S;
-      for (int hh = warp; hh < hper; hh += 8) {
-        const int h = (int)rank * hper + hh;
-        // (max, sum) of source split `lane`
-        float2 ml = make_float2(-INFINITY, 0.f);
-        if (lane < (int)S) ml = ld_peer_f2(peer_addr(tc::smem_u32(smem + OFF_SEL) + h * 8, (uint32_t)lane));
+    // ---- combine heads [rank * 128 / S, +128 / S) of this (row, half) from
+    // the partials every CTA of the cluster wrote before the barrier
+    cluster_sync_all();
+    const int S = a.splits;
+    const int hper = TH / S;
+    if (warp < 8) {
+      const int64_t slot0 = (int64_t)pair * S;
+      for (int hl = warp; hl < hper; hl += 8) {
+        const int h = split * hper + hl;
+        const float2 ml = lane < S ? __ldcg(a.ws_ml + (slot0 + lane) * TH + h) : make_float2(-INFINITY, 0.f);
+        // every source's row in flight before any use
+        float4 v0[8], v1[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (j < S) {
+            // d = 8 lane .. 8 lane + 7: block lane / 4, offset 8 (lane % 4)
+            const float4 *src = reinterpret_cast<const float4 *>(
+                a.ws_o + (slot0 + j) * TH * DHALF + ((int64_t)(lane >> 2) * TH + h) * 32 + (lane & 3) * 8);
+            v0[j] = __ldcg(src);
+            v1[j] = __ldcg(src + 1);
+          }
+        }
         float M = ml.x;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -523,26 +475,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
         float L = wgt * ml.y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        // all sources' loads in flight before any use
-        float wj[8];
-        float4 v0[8], v1[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          wj[j] = __shfl_sync(0xffffffffu, wgt, j);
-          v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < (int)S && wj[j] != 0.f) {
-            const uint32_t base = peer_addr(tc::smem_u32(smem + OFF_Q), (uint32_t)j);
-            v0[j] = ld_peer_f4(base + po_off(h, 2 * lane));
-            v1[j] = ld_peer_f4(base + po_off(h, 2 * lane + 1));
-          }
-        }
         float acc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          acc[0] += wj[j] * v0[j].x; acc[1] += wj[j] * v0[j].y; acc[2] += wj[j] * v0[j].z; acc[3] += wj[j] * v0[j].w;
-          acc[4] += wj[j] * v1[j].x; acc[5] += wj[j] * v1[j].y; acc[6] += wj[j] * v1[j].z; acc[7] += wj[j] * v1[j].w;
+          const float wj = __shfl_sync(0xffffffffu, wgt, j);
+          acc[0] += wj * v0[j].x; acc[1] += wj * v0[j].y; acc[2] += wj * v0[j].z; acc[3] += wj * v0[j].w;
+          acc[4] += wj * v1[j].x; acc[5] += wj * v1[j].y; acc[6] += wj * v1[j].z; acc[7] += wj * v1[j].w;
         }
         const float inv = 1.f / L;
         uint32_t w[4];
@@ -556,12 +496,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const Args a) {
         if (a.lse && dh == 0 && lane == 0) a.lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
       }
     }
-    // this CTA's shared memory stays valid until every peer has finished reading it
-    __syncthreads();
-    if (tid == 0)
-      for (uint32_t r = 0; r < S; ++r) peer_arrive(peer_addr(tc::smem_u32(&bars[BAR_MDONE]), r));
-    if (tid == 0) wait_cluster_bar(&bars[BAR_MDONE], a.status);
-    __syncthreads();
   }
   if (warp == 8) tc::tmem_dealloc(tbase, TMEM_COLS);
 }
@@ -583,11 +517,17 @@ static void tc_plan(const csa_dims *d, bool dense, int *splits, int *cps) {
 
 bool attend_tc_supported(const csa_dims *d) { return d->H == TH && d->D == TD; }
 
-size_t attend_tc_workspace(const csa_dims *, bool) { return 0; }
+size_t attend_tc_workspace(const csa_dims *d, bool dense) {
+  int splits, cps;
+  tc_plan(d, dense, &splits, &cps);
+  if (splits == 1) return 0;
+  const int64_t slots = (int64_t)d->B * d->Tq * 2 * splits;
+  return (size_t)(slots * TH * (DHALF * 4 + 8)) + 256;
+}
 
 int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scales, const int32_t *idx,
                      const uint8_t *wcodes, const float *wscales, const int32_t *q_pos,
-                     const csa_dims *d, uint16_t *out, float *lse, void *,
+                     const csa_dims *d, uint16_t *out, float *lse, void *workspace,
                      cudaStream_t stream) {
   const bool dense = idx == nullptr;
   int splits, cps;
@@ -601,6 +541,11 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
   a.splits = splits; a.cps = cps;
   a.out = reinterpret_cast<__nv_bfloat16 *>(out);
   a.lse = lse;
+  const int64_t slots = rows * 2 * splits;
+  a.ws_o = splits > 1 ? static_cast<float *>(workspace) : nullptr;
+  a.ws_ml = splits > 1 ? reinterpret_cast<float2 *>(static_cast<char *>(workspace) + (size_t)(slots * TH * DHALF * 4))
+                       : nullptr;
+  if (splits > 1 && !workspace) return fail(CSA_ERR_WORKSPACE, "attend: workspace required");
   a.status = status_word_device_ptr();
   if (int rc = set_smem_once((const void *)attend_tc_kernel, (int)SMEM_BYTES, "attend_tc_kernel")) return rc;
   const int64_t grid = rows * 2 * splits;
@@ -617,7 +562,12 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, a);
+  // Q viewed as [rows * 128 heads][512 d] bf16; boxes of 16 d x 128 heads
+  CUtensorMap qmap;
+  if (!encode_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, TD, (uint64_t)(rows * TH), TD * 2, 16, TH,
+                      CU_TENSOR_MAP_SWIZZLE_32B))
+    return fail(CSA_ERR_INVALID, "attend: cannot map the queries for TMA (misaligned?)");
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, qmap, a);
   count_launches(1);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attend_tc_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("attend_tc_kernel");

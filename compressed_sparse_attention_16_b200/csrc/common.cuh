@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -32,6 +33,11 @@ unsigned *status_word_device_ptr();   // address of the status word, current dev
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel), so
 // that launches captured into CUDA graphs issue no attribute calls.
 int set_smem_once(const void *kernel, int bytes, const char *name);
+// 2-D tensor map for TMA loads: `rows` rows of `inner` elements, `row_bytes`
+// apart; boxes of box_inner x box_rows.  False if the driver entry point is
+// missing or the encoder rejects the arguments.
+bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner, uint64_t rows,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 __device__ __forceinline__ void raise_status(unsigned *status, unsigned bit) {
   atomicOr(status, bit);

@@ -21,8 +21,6 @@
 // radix select (12 bits per digit) over a shared-memory histogram, ties at
 // the threshold are resolved by index, and the K survivors are sorted with a
 // bitonic network.
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -1436,24 +1434,10 @@ size_t fd_workspace(const csa_dims *d, int per_row, FdWs *ws, void *base, size_t
 // Tensor map over the indexer keys viewed as [B * entry_cap rows][32 bytes],
 // 256-row boxes, 32-byte swizzle (the layout the MMA descriptor reads).
 bool fd_key_map(const uint8_t *kI, const csa_dims *d, CUtensorMap *map) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  if (!encode) {
-    void *fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn)
-      return false;
-    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
   const int64_t rows = (int64_t)d->B * d->entry_cap;
-  if (((uintptr_t)kI & 15u) != 0 || rows < 1 || rows >= (1ll << 31)) return false;
-  const cuuint64_t dims[2] = {32, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {32};
-  const cuuint32_t box[2] = {32, 256};
-  const cuuint32_t estr[2] = {1, 1};
-  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(kI), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (rows >= (1ll << 31)) return false;
+  return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, kI, 32, (uint64_t)rows, 32, 32, 256,
+                        CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 int launch_fd(const CUtensorMap &kmap, const uint8_t *qI, const float *w, const int32_t *q_pos, const csa_dims *d,
