@@ -167,6 +167,7 @@ class Runner:
         self.dev = device
         torch.cuda.set_device(device)
         self.graphs = {}
+        self._side = None
         self.decode = wl.kind in ("decode", "decode_incremental", "hca_decode")
         if self.decode:
             self.n_new = wl.m if wl.kind == "hca_decode" else 4
@@ -299,6 +300,27 @@ class Runner:
         for _, fn in self.calls(i, inputs):
             fn()
 
+    def _capture_step(self, calls):
+        """Issue one step's calls as a fork/join: the appends (compress) feed
+        only the attention, so they run on a side stream beside the indexer
+        (CSA) or beside each other (HCA); the attention waits for both."""
+        torch = self.torch
+        if self._side is None:
+            self._side = torch.cuda.Stream(device=self.dev)
+        side, main = self._side, torch.cuda.current_stream(self.dev)
+        appends = [fn for name, fn in calls if name.startswith("compress")]
+        index = [fn for name, fn in calls if name == "index_topk"]
+        final = [fn for name, fn in calls if not name.startswith("compress") and name != "index_topk"]
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            for fn in (appends if index else appends[1:]):
+                fn()
+        for fn in (index if index else appends[:1]):
+            fn()
+        main.wait_stream(side)
+        for fn in final:
+            fn()
+
     def graph(self, i, inputs=None, key=None):
         """CUDA graph of step i (captured once)."""
         import compressed_sparse_attention_16_b200 as csa
@@ -315,11 +337,27 @@ class Runner:
             g = torch.cuda.CUDAGraph()
             n0 = csa.launch_count()
             with torch.cuda.graph(g):
-                for _, fn in calls:
-                    fn()
+                self._capture_step(calls)
             g.kernels = csa.launch_count() - n0
             self.graphs[key] = g
         return g
+
+
+def max_over_ranks(ms, world, device):
+    """The job's duration: the maximum of one per-rank duration over all ranks
+    (an all-reduce on the default process group when world > 1)."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank, ms):
+    """Whole-job units per second: every rank processes its own units (weak
+    scaling) in at most `ms` milliseconds."""
+    return world * units_per_rank / (ms / 1e3)
 
 
 def l2_flush(buf):
@@ -390,13 +428,9 @@ def gpu_arm(args, wl):
     barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
-    step_ms = float(sum(a.elapsed_time(b) for a, b in step_events))
-    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms = float(t.item())
+    step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_events), world, dev)
     ms_per_step = step_ms / args.steps
-    value = world * r.units_per_step / (ms_per_step / 1e3)
+    value = job_throughput(world, r.units_per_step, ms_per_step)
 
     # per-call device time: each call alone, cold L2, queued behind a bounded sleep
     per_call = {}
@@ -491,13 +525,8 @@ def e2e_leg(r, args, world, dev, use_graph):
         torch.cuda.synchronize()
         if i >= 2:
             times.append(e0.elapsed_time(e1))
-    ms = float(np.mean(times))
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": world * r.units_per_step / (ms / 1e3), "unit": r.unit,
+    ms = max_over_ranks(np.mean(times), world, dev)
+    return {"value": job_throughput(world, r.units_per_step, ms), "unit": r.unit,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 

@@ -38,6 +38,7 @@ SYMBOLS = (
     "csa_sync_status",
     "csa_version",
     "csa_launch_count",
+    "csa_selftest_timeout",
 )
 
 
@@ -104,6 +105,8 @@ def lib() -> ctypes.CDLL:
     L.csa_version.restype = ctypes.c_int
     L.csa_launch_count.argtypes = []
     L.csa_launch_count.restype = ctypes.c_uint64
+    L.csa_selftest_timeout.argtypes = [ctypes.c_uint64, _P]
+    L.csa_selftest_timeout.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -240,6 +243,12 @@ def sync_status(stream=None) -> None:
 
 def version() -> int:
     return int(lib().csa_version())
+
+
+def selftest_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Run the bounded-wait diagnostic kernel (its wait always expires); the
+    next sync_status() raises CsaError(CSA_ERR_TIMEOUT)."""
+    _check(lib().csa_selftest_timeout(int(limit_ns), _stream(stream)))
 
 
 def launch_count() -> int:

@@ -105,6 +105,34 @@ int set_smem_once(const void *kernel, int bytes, const char *name) {
   return fail(CSA_ERR_CUDA, "%s: attribute table full", name);
 }
 
+// A bounded wait on a phase nothing completes: it gives up after limit_ns
+// and reports STATUS_TIMEOUT, the path every pipeline wait takes on expiry.
+__global__ void selftest_timeout_kernel(unsigned long long limit_ns, unsigned *status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(1u) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    uint64_t t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
+      uint32_t ok;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(a), "r"(0u)
+          : "memory");
+      if (ok) break;   // never: no thread arrives
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > limit_ns) {
+        raise_status(status, STATUS_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
 }  // namespace csa
 
 using namespace csa;
@@ -143,6 +171,16 @@ extern "C" {
 int csa_version(void) { return 100; }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int csa_selftest_timeout(uint64_t limit_ns, csa_stream_t stream) {
+  csa::clear_error();
+  if (limit_ns < 1000ull) limit_ns = 1000ull;
+  if (limit_ns > 100000000ull) limit_ns = 100000000ull;
+  csa::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns,
+                                                                                 csa::status_word_device_ptr());
+  csa::count_launches(1);
+  return csa::check_launch("selftest_timeout_kernel");
+}
 
 const char *csa_last_error(void) { return g_err; }
 

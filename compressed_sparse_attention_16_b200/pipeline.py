@@ -98,6 +98,7 @@ class DecodeState:
         self.lse = torch.empty((B, 1, H), dtype=torch.float32, device=dev)
         self._ws_index = None
         self._ws_attend = None
+        self._side = None
 
     @property
     def n_entries(self) -> int:
@@ -139,9 +140,11 @@ class DecodeState:
             self.kI[:, first:first + n // self.m].copy_(kI_new)
         self.n_tokens += n
 
-    def query(self, q: torch.Tensor, qI: torch.Tensor | None = None, w: torch.Tensor | None = None):
+    def query(self, q: torch.Tensor, qI: torch.Tensor | None = None, w: torch.Tensor | None = None,
+              after: torch.cuda.Stream | None = None):
         """One query per sequence at position n_tokens - 1.  q: bf16 [B, 1, H, D];
-        qI: u8 [B, 1, HI, dI/2], w: f32 [B, 1, HI] (CSA only)."""
+        qI: u8 [B, 1, HI, dI/2], w: f32 [B, 1, HI] (CSA only).  The attention
+        waits for the stream `after` (if given)."""
         self.q_pos.fill_(self.n_tokens - 1)
         d = self.dims()
         if self.dense:
@@ -155,6 +158,8 @@ class DecodeState:
         if nb and (self._ws_index is None or self._ws_index.numel() < nb):
             self._ws_index = _ws(nb, self.device)
         index_topk(qI, w, self.kI, self.q_pos, d, self.idx, self.score, workspace=self._ws_index)
+        if after is not None:
+            torch.cuda.current_stream(self.device).wait_stream(after)
         nb = attend_workspace(d, False)
         if nb and (self._ws_attend is None or self._ws_attend.numel() < nb):
             self._ws_attend = _ws(nb, self.device)
@@ -163,6 +168,30 @@ class DecodeState:
         return self.out, self.lse
 
     def step(self, x_new, z_new, q, qI=None, w=None, kI_new=None):
-        """Append tokens then run one query per sequence at the newest position."""
-        self.append(x_new, z_new, kI_new)
-        return self.query(q, qI, w)
+        """Append tokens then run one query per sequence at the newest position.
+
+        CSA: the new entries' indexer keys are stored first; the compression
+        of the new tokens (needed only by the attention) runs on a side stream
+        beside the indexer, and the attention waits for both."""
+        if self.dense:
+            self.append(x_new, z_new, kI_new)
+            return self.query(q, qI, w)
+        main = torch.cuda.current_stream(self.device)
+        if self._side is None:
+            self._side = torch.cuda.Stream(device=self.device)
+        side = self._side
+        n = x_new.shape[1]
+        assert self.n_tokens % self.m == 0 and n % self.m == 0
+        first = self.n_entries
+        assert first + n // self.m <= self.entry_cap
+        if kI_new is not None and self.kI is not None:
+            self.kI[:, first:first + n // self.m].copy_(kI_new)
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            compress(x_new, z_new, self.m, self.codes, self.scales, dst_first=first)
+            compress(x_new, z_new, 1, self.win_codes, self.win_scales, dst_first=self.n_tokens,
+                     ring_cap=self.win_cap)
+        x_new.record_stream(side)
+        z_new.record_stream(side)
+        self.n_tokens += n
+        return self.query(q, qI, w, after=side)

@@ -219,6 +219,16 @@ const char *csa_last_error(void);
  */
 int csa_sync_status(csa_stream_t stream);
 
+/* Diagnostic of the failure path (no counterpart on the pages): launches one
+ * small kernel whose bounded wait is on an mbarrier phase that nothing
+ * completes.  After `limit_ns` nanoseconds of wall time (clamped to
+ * [1 us, 100 ms]) the wait gives up exactly as a stalled pipeline in the
+ * other kernels does: it sets the timeout bit in the device status word and
+ * the kernel returns, leaving the context usable.  The next
+ * csa_sync_status(stream) therefore returns CSA_ERR_TIMEOUT (and clears the
+ * bit).  Returns CSA_OK or CSA_ERR_CUDA if the launch fails. */
+int csa_selftest_timeout(uint64_t limit_ns, csa_stream_t stream);
+
 /* Library ABI version (major * 100 + minor). */
 int csa_version(void);
 

@@ -168,3 +168,20 @@ def test_prefill_128k_full_size_sampled():
         U = np.concatenate([_entry_values(x, z, 0, sel, wl.m), _window_values(x, 0, ocsa.window_positions(t, wl.W))])
         ro[0, i], rl[0, i] = ocsa.attend_one(qv[0, i], U)
     parity.check_attention(r.out[:, rr], r.lse[:, rr], ro, rl)
+
+
+def test_bounded_wait_expiry_is_reported_and_context_survives():
+    """A device wait that nothing satisfies gives up after its limit, sets the
+    timeout status, and the context stays usable for the next call."""
+    import compressed_sparse_attention_16_b200 as csa
+    csa.sync_status()
+    csa.selftest_timeout(2_000_000)
+    with pytest.raises(csa.CsaError) as e:
+        csa.sync_status()
+    assert e.value.code == csa.CSA_ERR_TIMEOUT
+    csa.sync_status()                        # the bit was cleared
+    x = torch.randn(1, 8, 64, device="cuda")
+    codes = torch.empty((1, 2, 64), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((1, 2), device="cuda")
+    csa.compress(x, torch.zeros_like(x), 4, codes, scales)
+    csa.sync_status()
