@@ -442,9 +442,13 @@ __device__ __forceinline__ void run_softmax(const PArgs &a, unsigned char *smem,
     if (it > 0) pwait(&bars[B_P2DONE], (it - 1) & 1, misc, a.status);
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
-      float mrow[32], sm[32];
+      // the shifted row maxima stay in shared memory (broadcast reads): fewer live registers
+      float *Ms = invL;                              // [64] free until the epilogue
+      if (hh == 0 && stid < PH) Ms[stid] = Mh[stid] + ri.eshift;
+      named_sync(2, kSoft);
+      float sm[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) { mrow[j] = Mh[hh * 32 + j] + ri.eshift; sm[j] = 0.f; }
+      for (int j = 0; j < 32; ++j) sm[j] = 0.f;
       for (int tl = 0; tl < ri.ntiles; ++tl) {
         uint32_t r[32];
         tc::tmem_ld32(tbase + lane_off + tl * PH + hh * 32, r);
@@ -456,8 +460,9 @@ __device__ __forceinline__ void run_softmax(const PArgs &a, unsigned char *smem,
         uint32_t pw[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const float pa = valid ? ex2(__uint_as_float(r[j]) * f - mrow[j]) : 0.f;
-          const float pb = valid ? ex2(__uint_as_float(r[j + 1]) * f - mrow[j + 1]) : 0.f;
+          const float2 mm = *reinterpret_cast<const float2 *>(Ms + hh * 32 + j);
+          const float pa = valid ? ex2(__uint_as_float(r[j]) * f - mm.x) : 0.f;
+          const float pb = valid ? ex2(__uint_as_float(r[j + 1]) * f - mm.y) : 0.f;
           sm[j] += pa;
           sm[j + 1] += pb;
           const __half2 v = __floats2half2_rn(pa * sc, pb * sc);
