@@ -9,28 +9,36 @@
 // 512 blocks per query, 128-token window.
 //
 // With only 64 heads per query the items fill the tensor core's M = 128
-// dimension instead:
-//   pass 1   S^T[item, head] = K_items . Q^T   (M = 128 items per tile,
-//            N = 64 heads, K = 512 in four 128-wide blocks); all <= 5 tiles of
-//            the row stay in TMEM (<= 320 columns);
-//   softmax  per head over items, i.e. across TMEM lanes: each warp reduces its
-//            32 lanes with a transposing butterfly, four quadrants combine in
-//            shared memory; P^T = p * entry scale is written as fp16;
-//   pass 2   O^T[d, head] = V^T . P^T  (M = 128 d per block, N = 64 heads,
-//            K = items), reading the same [item][d] tiles MN-major, one
-//            128-wide d block at a time into two alternating 64-column TMEM
-//            buffers;
+// dimension instead.  A row's items (<= 640) are processed in tiles of 128;
+// each tile is gathered and converted once and feeds both products:
+//   S^T[item, head] = K_tile . Q^T      (M = 128 items, N = 64 heads, K = 512)
+//   online softmax per head over the tile's items, i.e. across TMEM lanes:
+//            each warp reduces its 32 lanes with a transposing butterfly, the
+//            four quadrants combine in shared memory; the running maximum is
+//            raised lazily (only when a tile exceeds it by more than 2^8), and
+//            then O^T and the running sum are rescaled; P^T = p * entry scale
+//            is written as fp16;
+//   O^T[d, head] += V^T_tile . P^T      (M = 128 d per block, four blocks,
+//            N = 64 heads, K = 128 items), reading the same [item][d] tile
+//            MN-major; O^T for all 512 d stays in TMEM (256 columns);
 //   epilogue O / l straight from TMEM to the bf16 output rows.
+// The tile sits in shared memory as four 128 x 128 fp16 blocks, one slot per
+// 128-wide d block; a slot is refilled with the next tile's block as soon as
+// the MMAs of this tile's O^T block have read it.
 //
 // Roles (persistent CTAs, one per SM, query rows round-robin):
-//   warps 0-7   producers: per row, compact the selection into item row
-//               numbers and scales, convert Q, then gather every 128 x 128
-//               block of E4M3 codes (twice: once per pass) through registers,
-//               three blocks ahead, convert it exactly to fp16 and hand it to
-//               the tensor core through a two-slot shared-memory ring;
-//   warps 8-11  softmax of a row, then its epilogue (which overlaps pass 1 of
-//               the next row);
-//   warp 12     issues the MMAs (one thread) and commits them to mbarriers.
+//   warps 0-7   producers: gather every 128 x 128 block of E4M3 codes through
+//               registers, three blocks ahead (across rows), convert it
+//               exactly to fp16 and hand it to the tensor core;
+//   warps 8-11  softmax of each tile, then the row's epilogue (which overlaps
+//               the first scores of the next row);
+//   warp 12     issues the MMAs (one thread) and commits them to mbarriers;
+//   warps 13-14 per-row set-up, up to a row ahead: compact the selection
+//               into item row numbers and scales, the Q and scale maxima,
+//               then Q in fp16 once the previous row's scores are complete.
+// After the first tile of a row the softmax computes P^T against the running
+// maximum straight away and takes the separate maximum pass only when some
+// score exceeds it by more than 2^8.
 // Every wait is bounded; a wait that gives up raises STATUS_TIMEOUT and turns
 // every later wait of the CTA into a no-op, so all roles run to the end.
 //
@@ -39,10 +47,12 @@
 //   Q    one factor 2^kq per row puts max|q| in [2^14, 2^15): every bf16 value
 //        down to 2^-31 of the row maximum converts exactly; the factor is
 //        divided out of the scores in fp32;
-//   P^T  exp2(x - max_h - E), with the integer E chosen from the row's largest
-//        entry scale so that p * scale <= 2^15.  The same shift divides the
-//        softmax denominator, so O = sum(P^T v) / sum(p) needs no correction
-//        and the log-sum-exp adds E back.
+//   P^T  exp2(x - m_h - E), with the integer E chosen from the row's largest
+//        entry scale: the lazy maximum lets exp2(x - m_h) reach 2^8, and
+//        E = e - 133 for a largest scale below 2^(e - 126) keeps
+//        p * scale < 2^15.  The same shift divides the softmax denominator,
+//        so O = sum(P^T v) / sum(p) needs no correction and the log-sum-exp
+//        adds E back.
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -51,50 +61,60 @@ namespace {
 
 constexpr int PH = 64;             // heads (MMA N)
 constexpr int PD = 512;            // entry width
-constexpr int PT = 128;            // items per tile (MMA M of pass 1)
+constexpr int PT = 128;            // items per tile (MMA M of the scores)
 constexpr int PDB = 128;           // d per block
+constexpr int kNdb = PD / PDB;     // d blocks (= ring slots)
 constexpr int kMaxTiles = 5;       // <= 640 items per row
 constexpr int kMaxItems = kMaxTiles * PT;
 constexpr int kProd = 256;         // producer threads (warps 0-7)
 constexpr int kSoft = 128;         // softmax / epilogue threads (warps 8-11)
-constexpr int kThreads = kProd + kSoft + 32;
+constexpr int kSetup = 64;         // set-up threads (warps 13-14)
 constexpr int kMmaWarp = (kProd + kSoft) / 32;
+constexpr int kSetupWarp0 = kMmaWarp + 1;
+constexpr int kThreads = kProd + kSoft + 32 + kSetup;
 constexpr float kPLog2e = 1.4426950408889634f;
+constexpr float kPRescaleLog2 = 8.f;
 constexpr unsigned long long kPWaitNs = 2000000000ull;
-constexpr uint32_t kOCol = kMaxTiles * PH;   // O^T buffers: columns [320, 448)
+constexpr uint32_t kSCol = 0;      // S^T: TMEM columns [0, 64)
+constexpr uint32_t kOCol = PH;     // O^T: four blocks of 64 columns, [64, 320)
 
 // shared memory map (bytes)
 constexpr uint32_t S_Q = 0;                                  // fp16 [64 h][512 d]          64 KiB
-constexpr uint32_t S_PT = S_Q + PH * PD * 2;                 // fp16 [640 i][64 h]          80 KiB
-constexpr uint32_t S_KV = S_PT + kMaxItems * PH * 2;         // fp16 2 x [128 i][128 d]     64 KiB
+constexpr uint32_t S_PT = S_Q + PH * PD * 2;                 // fp16 [128 i][64 h]          16 KiB
+constexpr uint32_t S_KV = S_PT + PT * PH * 2;                // fp16 4 x [128 i][128 d]    128 KiB
 constexpr uint32_t KV_BYTES = PT * PDB * 2;
-constexpr uint32_t S_ITEM = S_KV + 2 * KV_BYTES;             // int32 [2][640] item rows
+constexpr uint32_t S_ITEM = S_KV + kNdb * KV_BYTES;          // int32 [2][640] item rows
 constexpr uint32_t S_SCALE = S_ITEM + 2 * kMaxItems * 4;     // fp32 [2][640] item scales
 constexpr uint32_t S_INFO = S_SCALE + 2 * kMaxItems * 4;     // RowInfo [2]
-constexpr uint32_t S_RED = S_INFO + 2 * 32;                  // fp32 [4][64], M[64], L[64], 1/L[64]
-constexpr uint32_t S_PRED = S_RED + 8 * PH * 4;              // producer reductions, u32 [16]
-constexpr uint32_t S_BAR = S_PRED + 16 * 4;
-constexpr int kNumBars = 16;
+constexpr uint32_t S_RED = S_INFO + 2 * 32;                  // fp32: max [4][64], sum [4][64], M, L, Ms, invL, fac [64]
+constexpr uint32_t S_PRED = S_RED + 13 * PH * 4;             // set-up reductions, u32 [16]
+constexpr uint32_t S_FLAG = S_PRED + 16 * 4;                 // int [2] rescale, int [2] slow path
+constexpr uint32_t S_BAR = S_FLAG + 16;
+constexpr int kNumBars = 20;
 constexpr uint32_t S_MISC = S_BAR + kNumBars * 8;
 constexpr uint32_t P_SMEM = S_MISC + 32;
 static_assert(P_SMEM <= 232448, "shared memory");
+static_assert(S_KV % 1024 == 0 && S_PT % 1024 == 0, "tile alignment");
 
 // mbarriers
 enum : int {
-  B_FULL = 0,      // [2] producers -> MMA: ring slot converted (one arrival per warp)
-  B_EMPTY = 2,     // [2] MMA -> producers: ring slot read (commit)
-  B_READY = 4,     // [2] producers -> all: row set-up done, by row parity (one per warp)
-  B_P1DONE = 6,    // MMA -> softmax, producers: S^T complete, Q no longer read (commit)
-  B_PTFULL = 7,    // softmax -> MMA: P^T written, S^T read (1 arrival)
-  B_P2DONE = 8,    // MMA -> softmax: P^T no longer read (commit)
-  B_OFULL = 9,     // [2] MMA -> epilogue: O^T buffer complete (commit)
-  B_OEMPTY = 11,   // [2] epilogue -> MMA: O^T buffer read (one arrival per warp)
-  B_FINAL = 13,    // all MMAs complete (commit)
+  B_FULL = 0,      // [4] producers -> MMA: d-block slot converted (one arrival per warp)
+  B_EMPTY = 4,     // [4] MMA -> producers: d-block slot read by the tile's last MMA (commit)
+  B_READY = 8,     // [2] set-up -> softmax, MMA: RowInfo and Q in place, by row parity (one per warp)
+  B_ITEMS = 10,    // [2] set-up -> producers: item rows in place, by row parity (one per warp)
+  B_FREE = 12,     // [2] producers (one per warp) + softmax (one) -> set-up: the row's item
+                   //     rows and scales are no longer read
+  B_QFREE = 14,    // MMA -> set-up: the row's last scores complete, Q no longer read (commit)
+  B_SFULL = 15,    // MMA -> softmax: S^T of a tile complete (commit)
+  B_PFULL = 16,    // softmax -> MMA: P^T written, S^T read, O^T rescaled (1 arrival)
+  B_OFULL = 17,    // MMA -> epilogue: the row's O^T complete (commit)
+  B_OEMPTY = 18,   // epilogue -> MMA: O^T read (one arrival per warp)
+  B_FINAL = 19,    // all MMAs complete (commit)
 };
 
 // Q  [64 h][512 d]:   d-group stride 1024, head-group stride 128
 // KV [128 i][128 d]:  d-group stride 2048, item-group stride 128
-// PT [640 i][64 h]:   item-group stride 1024, head-group stride 128
+// PT [128 i][64 h]:   item-group stride 1024, head-group stride 128
 __device__ __forceinline__ uint32_t pq_off(int h, int g) { return g * 1024 + (h >> 3) * 128 + (h & 7) * 16; }
 __device__ __forceinline__ uint32_t pkv_off(int i, int g) { return g * 2048 + (i >> 3) * 128 + (i & 7) * 16; }
 __device__ __forceinline__ uint32_t ppt_off(int i, int hg) { return (i >> 3) * 1024 + hg * 128 + (i & 7) * 16; }
@@ -202,136 +222,166 @@ struct PArgs {
   unsigned *status;
 };
 
-// ------------------------------------------------------------------ producers
-// The producers walk one stream of blocks over all rows of the CTA.  Row it
-// has nbt = 8 * ntiles blocks: j < nb1 = 4 * ntiles is pass 1, tile j / 4, d
-// block j % 4; j = nb1 + jj is pass 2, d block jj / ntiles, tile jj % ntiles.
-// Blocks are gathered into registers three ahead of the one being converted
-// (across row boundaries); the set-up of row it + 1 (selection, scales, Q)
-// runs once pass 1 of row it has been handed over, while the softmax of row it
-// keeps the tensor core waiting anyway.
-__device__ __forceinline__ void run_producers(const PArgs &a, unsigned char *smem, int nrows) {
+// ------------------------------------------------------------------- set-up
+// Row it uses the item, scale and RowInfo buffers of parity it & 1; they are
+// rewritten for row it + 2 once the producers have gathered row it's last
+// block and the softmax has used row it's last scales (B_FREE).
+__device__ __forceinline__ void run_setup(const PArgs &a, unsigned char *smem, int nrows) {
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S_BAR);
   PMisc *misc = reinterpret_cast<PMisc *>(smem + S_MISC);
   RowInfo *info = reinterpret_cast<RowInfo *>(smem + S_INFO);
   uint32_t *pred = reinterpret_cast<uint32_t *>(smem + S_PRED);
-  const int tid = threadIdx.x, pw = tid >> 5, lane = tid & 31;
-  const int i8 = lane & 7, cq = lane >> 3;
+  const int st = threadIdx.x - kSetupWarp0 * 32, sw = st >> 5, lane = threadIdx.x & 31;
   const float qs = a.sm_scale * kPLog2e;
-  int ni0 = 0, ni1 = 0, nt0 = 0, nt1 = 0;   // n_items / ntiles of the rows of parity 0 / 1
 
-  // ---- per-row set-up: item rows and scales, Q in fp16, RowInfo
-  auto setup = [&](int it) {
+  for (int it = 0; it < nrows; ++it) {
     const int row = blockIdx.x + it * gridDim.x;
     const int par = it & 1;
+    if (it >= 2) pwait(&bars[B_FREE + par], ((it >> 1) - 1) & 1, misc, a.status);
     int *irow = reinterpret_cast<int *>(smem + S_ITEM) + par * kMaxItems;
     float *isc = reinterpret_cast<float *>(smem + S_SCALE) + par * kMaxItems;
     const int b = row / a.Tq;
     int64_t t = a.q_pos[row];
     if (t < 0) {
-      if (tid == 0) raise_status(a.status, STATUS_BAD_POSITION);
+      if (st == 0) raise_status(a.status, STATUS_BAD_POSITION);
       t = 0;
     }
     const int nwin = (int)min((int64_t)a.W, t + 1);
     const int64_t p0 = t - nwin + 1;
     // ordered compaction of the valid selected entries into item rows:
-    // r >= 0 is row r of the entry cache, r < 0 row -r-1 of the window ring
+    // r >= 0 is row r of the entry cache, r < 0 row -r-1 of the window ring.
+    // The indices are read eight per thread up front, so that their loads
+    // (and the scale loads they lead to) overlap.
     const int32_t *idx = a.idx + (int64_t)row * a.K;
+    constexpr int kPer = 8;
     int nsel = 0;
-    for (int j0 = 0; j0 < a.K; j0 += kProd) {
-      const int j = j0 + tid;
-      int e = (j < a.K) ? idx[j] : -1;
-      if (e >= a.n_entries || e < -1) { raise_status(a.status, STATUS_BAD_INDEX); e = -1; }
-      const bool f = e >= 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
-      if (lane == 0) pred[pw] = __popc(bal);
-      named_sync(1, kProd);
-      int before = 0, tot = 0;
+    for (int j0 = 0; j0 < a.K; j0 += kSetup * kPer) {
+      int e[kPer];
 #pragma unroll
-      for (int k = 0; k < kProd / 32; ++k) {
-        const int c = (int)pred[k];
-        before += (k < pw) ? c : 0;
-        tot += c;
+      for (int k = 0; k < kPer; ++k) {
+        const int j = j0 + k * kSetup + st;
+        e[k] = (j < a.K) ? idx[j] : -1;
       }
-      if (f) {
-        const int u = nsel + before + __popc(bal & ((1u << lane) - 1u));
-        const int64_t r = (int64_t)b * a.entry_cap + e;
-        irow[u] = (int)r;
-        isc[u] = a.scales[r];
+      float sv[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        if (e[k] >= a.n_entries || e[k] < -1) { raise_status(a.status, STATUS_BAD_INDEX); e[k] = -1; }
+        sv[k] = e[k] >= 0 ? a.scales[(int64_t)b * a.entry_cap + e[k]] : 0.f;
       }
-      nsel += tot;
-      named_sync(1, kProd);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const bool f = e[k] >= 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) pred[2 * k + sw] = __popc(bal);
+      }
+      named_sync(3, kSetup);
+      int base = nsel;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const bool f = e[k] >= 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        const int c0 = (int)pred[2 * k], c1 = (int)pred[2 * k + 1];
+        if (f) {
+          const int u = base + (sw ? c0 : 0) + __popc(bal & ((1u << lane) - 1u));
+          irow[u] = (int)((int64_t)b * a.entry_cap + e[k]);
+          isc[u] = sv[k];
+        }
+        base += c0 + c1;
+      }
+      nsel = base;
+      named_sync(3, kSetup);
     }
     const int n_items = min(nsel + nwin, kMaxItems);
-    for (int u = nsel + tid; u < n_items; u += kProd) {
+    for (int u = nsel + st; u < n_items; u += kSetup) {
       const int64_t r = (int64_t)b * a.win_cap + (p0 + (u - nsel)) % a.win_cap;
       irow[u] = (int)(-r - 1);
       isc[u] = a.wscales[r];
     }
     const int ntiles = (n_items + PT - 1) / PT;
-    if (par) { ni1 = n_items; nt1 = ntiles; } else { ni0 = n_items; nt0 = ntiles; }
-    named_sync(1, kProd);
+    named_sync(3, kSetup);
+    // the producers may gather this row now
+    __syncwarp();
+    if (lane == 0) {
+      if (sw == 0) {
+        info[par].n_items = n_items;
+        info[par].ntiles = ntiles;
+      }
+    }
+    named_sync(3, kSetup);
+    if (lane == 0) tc::mbar_arrive(&bars[B_ITEMS + par]);
 
-    // Q: thread (pw, lane) holds head (lane & 7) + 8 pw, d-groups (lane >> 3) + 4 k;
-    // read twice (max, then convert) to keep few registers live
-    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * PH * PD);
-    const int h = i8 + 8 * pw;
+    // Q row max (thread st holds head st) and the largest scale
+    const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * PH * PD) + st * (PD / 8);
     uint32_t mq = 0;
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const uint4 v = __ldg(qg + h * (PD / 8) + cq + 4 * k);
+#pragma unroll 8
+    for (int k = 0; k < PD / 8; ++k) {
+      const uint4 v = __ldg(qg + k);
       mq = __vmaxu2(mq, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
                                  __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
     }
     float smax = 0.f;
-    for (int u = tid; u < n_items; u += kProd) smax = fmaxf(smax, isc[u]);
+    for (int u = st; u < n_items; u += kSetup) smax = fmaxf(smax, isc[u]);
     mq = __reduce_max_sync(0xffffffffu, max(mq & 0xFFFFu, mq >> 16));
     const uint32_t sbits = __reduce_max_sync(0xffffffffu, __float_as_uint(smax));   // smax >= 0
-    if (lane == 0) { pred[pw] = mq; pred[8 + pw] = sbits; }
-    named_sync(1, kProd);
-    uint32_t amax = 0, smb = 0;
-#pragma unroll
-    for (int k = 0; k < kProd / 32; ++k) { amax = max(amax, pred[k]); smb = max(smb, pred[8 + k]); }
+    if (lane == 0) { pred[sw] = mq; pred[8 + sw] = sbits; }
+    named_sync(3, kSetup);
+    const uint32_t amax = max(pred[0], pred[1]), smb = max(pred[8], pred[9]);
     // bf16 |q| max in [2^(eb-127), 2^(eb-126)) -> times 2^(141-eb) in [2^14, 2^15)
     const int kq = amax ? min(126, 141 - (int)((amax >> 7) & 0xFFu)) : 0;
     const float fq = __int_as_float((kq + 127) << 23);
-    if (tid == 0) {
-      RowInfo ri;
-      ri.row = row; ri.n_items = n_items; ri.ntiles = ntiles; ri.pad0 = 0;
+    if (st == 0) {
+      RowInfo &ri = info[par];
+      ri.row = row;
+      ri.pad0 = 0;
       ri.qscale = qs * __int_as_float((127 - kq) << 23);
-      // largest scale < 2^(e - 126) for biased exponent e; p * scale * 2^-E <= 2^15
+      // largest scale < 2^(e - 126) for biased exponent e; p <= 2^8 under the
+      // lazy maximum, so p * scale * 2^-E < 2^15 with E = e - 133
       const int e = (int)((smb >> 23) & 0xFFu);
-      ri.eshift = (float)min(104, max(-110, e - 141));
+      ri.eshift = (float)min(112, max(-110, e - 133));
       ri.pad1[0] = ri.pad1[1] = 0.f;
-      info[par] = ri;
     }
-    // the Q buffer is free once pass 1 of the previous row is complete
-    if (it > 0) pwait(&bars[B_P1DONE], (it - 1) & 1, misc, a.status);
+    // Q in fp16: the buffer is free once the previous row's last scores are complete
+    if (it > 0) pwait(&bars[B_QFREE], (it - 1) & 1, misc, a.status);
     unsigned char *qs_ = smem + S_Q;
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const uint4 v = __ldg(qg + h * (PD / 8) + cq + 4 * k);
-      *reinterpret_cast<uint4 *>(qs_ + pq_off(h, cq + 4 * k)) =
+#pragma unroll 8
+    for (int k = 0; k < PD / 8; ++k) {
+      const uint4 v = __ldg(qg + k);
+      *reinterpret_cast<uint4 *>(qs_ + pq_off(st, k)) =
           make_uint4(bf2_to_h2(v.x, fq), bf2_to_h2(v.y, fq), bf2_to_h2(v.z, fq), bf2_to_h2(v.w, fq));
     }
     tc::fence_proxy_async_smem();
-    __syncwarp();
+    // pred is reused by the next row
+    named_sync(3, kSetup);
     if (lane == 0) tc::mbar_arrive(&bars[B_READY + par]);
+  }
+}
+
+// ------------------------------------------------------------------ producers
+// The producers walk one stream of blocks over all rows of the CTA.  Row it
+// has 4 * ntiles blocks: block j is tile j / 4, d block j % 4, and goes to
+// ring slot j % 4.  Blocks are gathered into registers three ahead of the one
+// being converted, across row boundaries.
+__device__ __forceinline__ void run_producers(const PArgs &a, unsigned char *smem, int nrows) {
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S_BAR);
+  PMisc *misc = reinterpret_cast<PMisc *>(smem + S_MISC);
+  const RowInfo *info = reinterpret_cast<const RowInfo *>(smem + S_INFO);
+  const int tid = threadIdx.x, pw = tid >> 5, lane = tid & 31;
+  const int i8 = lane & 7, cq = lane >> 3;
+  int ni0 = 0, ni1 = 0, nt0 = 0, nt1 = 0;   // n_items / ntiles of the rows of parity 0 / 1
+
+  auto row_items = [&](int it) {
+    const int par = it & 1;
+    pwait(&bars[B_ITEMS + par], (it >> 1) & 1, misc, a.status);
+    const int n = info[par].n_items, t = info[par].ntiles;
+    if (par) { ni1 = n; nt1 = t; } else { ni0 = n; nt0 = t; }
   };
 
   // ---- block gather: thread (pw, lane) holds items (2 pw + (k & 1)) * 8 +
   // (lane & 7) of the tile, 16-byte chunks (k >> 1) * 4 + (lane >> 3) of the
   // d block, k = 0..3.  Items past n_items read item 0 (always valid): their
   // scores are masked and their P^T rows are zero.
-  auto block_of = [&](int it, int j, int &tile, int &dblk) {
-    const int ntiles = (it & 1) ? nt1 : nt0;
-    const int nb1 = ntiles * (PD / PDB);
-    if (j < nb1) { tile = j >> 2; dblk = j & 3; }
-    else { const int jj = j - nb1; dblk = jj / ntiles; tile = jj - dblk * ntiles; }
-  };
   auto load_blk = [&](int it, int j, uint4 (&v)[4]) {
-    int tile, dblk;
-    block_of(it, j, tile, dblk);
+    const int tile = j >> 2, dblk = j & 3;
     const int n_items = (it & 1) ? ni1 : ni0;
     const int *irow = reinterpret_cast<const int *>(smem + S_ITEM) + (it & 1) * kMaxItems;
 #pragma unroll
@@ -343,9 +393,9 @@ __device__ __forceinline__ void run_producers(const PArgs &a, unsigned char *sme
       v[k] = __ldg(reinterpret_cast<const uint4 *>(base + dblk * PDB + ((k >> 1) * 4 + cq) * 16));
     }
   };
-  uint32_t nblk = 0;   // blocks handed over so far (ring slot = nblk & 1)
+  uint32_t nblk = 0;   // blocks handed over so far (ring slot = nblk & 3 = d block)
   auto produce = [&](const uint4 (&v)[4]) {
-    const uint32_t slot = nblk & 1u, use = nblk >> 1;
+    const uint32_t slot = nblk & 3u, use = nblk >> 2;
     if (use > 0 && lane == 0) pwait(&bars[B_EMPTY + slot], (use - 1) & 1u, misc, a.status);
     __syncwarp();
     unsigned char *kv = smem + S_KV + slot * KV_BYTES;
@@ -364,28 +414,35 @@ __device__ __forceinline__ void run_producers(const PArgs &a, unsigned char *sme
     if (lane == 0) tc::mbar_arrive(&bars[B_FULL + slot]);
     ++nblk;
   };
-  auto nbt_of = [&](int it) { return ((it & 1) ? nt1 : nt0) * 2 * (PD / PDB); };
+  auto nbt_of = [&](int it) { return ((it & 1) ? nt1 : nt0) * kNdb; };
 
   if (nrows <= 0) return;
-  setup(0);
   int p_it = 0, p_j = 0;   // next block to hand over
   int l_it = 0, l_j = 0;   // next block to gather
+  auto gather = [&](uint4 (&v)[4]) {
+    if (l_it < nrows) {
+      if (l_j == 0) row_items(l_it);
+      load_blk(l_it, l_j, v);
+      if (++l_j == nbt_of(l_it)) {
+        // this row's item rows are no longer read by the producers
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars[B_FREE + (l_it & 1)]);
+        ++l_it;
+        l_j = 0;
+      }
+    }
+  };
   auto step = [&](uint4 (&v)[4]) {
     if (p_it < nrows) {
-      if (p_j == nbt_of(p_it) / 2 && p_it + 1 < nrows) setup(p_it + 1);
       produce(v);
       if (++p_j == nbt_of(p_it)) { ++p_it; p_j = 0; }
     }
-    if (l_it < nrows) {
-      load_blk(l_it, l_j, v);
-      if (++l_j == nbt_of(l_it)) { ++l_it; l_j = 0; }
-    }
+    gather(v);
   };
   uint4 A[4], B[4], C[4];
-  load_blk(0, 0, A);
-  load_blk(0, 1, B);
-  load_blk(0, 2, C);
-  l_j = 3;   // a row has at least 8 blocks
+  gather(A);
+  gather(B);
+  gather(C);
   while (p_it < nrows) {
     step(A);
     step(B);
@@ -398,116 +455,165 @@ __device__ __forceinline__ void run_softmax(const PArgs &a, unsigned char *smem,
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S_BAR);
   PMisc *misc = reinterpret_cast<PMisc *>(smem + S_MISC);
   const RowInfo *info = reinterpret_cast<const RowInfo *>(smem + S_INFO);
-  float *red = reinterpret_cast<float *>(smem + S_RED);   // [4][64]
-  float *Mh = red + 4 * PH;
-  float *Lh = Mh + PH;
-  float *invL = Lh + PH;
+  float *redm = reinterpret_cast<float *>(smem + S_RED);   // [4][64] tile maxima per quadrant
+  float *reds = redm + 4 * PH;                              // [4][64] tile sums per quadrant
+  float *Mh = reds + 4 * PH;                                // running maximum
+  float *Lh = Mh + PH;                                      // running sum
+  float *Ms = Lh + PH;                                      // running maximum + E
+  float *invL = Ms + PH;
+  float *fac = invL + PH;                                   // rescale factor of this tile
+  int *flag = reinterpret_cast<int *>(smem + S_FLAG);       // [2] rescale O^T
+  int *slow = flag + 2;                                     // [2] the running maximum is too low
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sq = warp - kProd / 32;        // TMEM lane quadrant
   const int stid = tid - kProd;
   const uint32_t lane_off = (uint32_t)(sq * 32) << 16;
-  uint32_t ouse = 0;
+  uint32_t ntile = 0;                      // tiles processed by this CTA
 
   for (int it = 0; it < nrows; ++it) {
     const int par = it & 1;
     pwait(&bars[B_READY + par], (it >> 1) & 1, misc, a.status);
     const RowInfo ri = info[par];
     const float *isc = reinterpret_cast<const float *>(smem + S_SCALE) + par * kMaxItems;
-    pwait(&bars[B_P1DONE], it & 1, misc, a.status);
-    tc::fence_after_sync();
+    // exp2(x - m) <= 2^8 <=> (x - m - E) <= 8 - E
+    const float thr = kPRescaleLog2 - ri.eshift;
+    if (stid < PH) { Mh[stid] = -INFINITY; Lh[stid] = 0.f; }
 
-    // max over items of x = score * scale * log2(e), per head
-#pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
-      float mx[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) mx[j] = -INFINITY;
-      for (int tl = 0; tl < ri.ntiles; ++tl) {
-        uint32_t r[32];
-        tc::tmem_ld32(tbase + lane_off + tl * PH + hh * 32, r);
-        tc::tmem_wait_ld();
-        const int u = tl * PT + sq * 32 + lane;
-        const bool valid = u < ri.n_items;
-        const float f = valid ? isc[u] * ri.qscale : 0.f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mx[j] = fmaxf(mx[j], valid ? __uint_as_float(r[j]) * f : -INFINITY);
-      }
-      red[sq * PH + hh * 32 + lane] = warp_transpose_reduce<true>(mx);
-    }
-    named_sync(2, kSoft);
-    if (stid < PH) Mh[stid] = fmaxf(fmaxf(red[stid], red[PH + stid]), fmaxf(red[2 * PH + stid], red[3 * PH + stid]));
-    named_sync(2, kSoft);
+    for (int tl = 0; tl < ri.ntiles; ++tl, ++ntile) {
+      pwait(&bars[B_SFULL], ntile & 1, misc, a.status);
+      tc::fence_after_sync();
+      const int u = tl * PT + sq * 32 + lane;
+      const bool valid = u < ri.n_items;
+      const float sc = valid ? isc[u] : 0.f;
+      const float f = sc * ri.qscale;
 
-    // P^T may be overwritten once pass 2 of the previous row is complete
-    if (it > 0) pwait(&bars[B_P2DONE], (it - 1) & 1, misc, a.status);
+      // P^T = exp2(x - m - E) * scale and the tile's sums of exp2(x - m - E);
+      // with `detect`, report any item whose exp2(x - m) would exceed 2^8
+      auto p_phase = [&](bool detect) {
+        bool over = false;
 #pragma unroll 1
-    for (int hh = 0; hh < 2; ++hh) {
-      // the shifted row maxima stay in shared memory (broadcast reads): fewer live registers
-      float *Ms = invL;                              // [64] free until the epilogue
-      if (hh == 0 && stid < PH) Ms[stid] = Mh[stid] + ri.eshift;
-      named_sync(2, kSoft);
-      float sm[32];
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r[32];
+          tc::tmem_ld32(tbase + lane_off + kSCol + hh * 32, r);
+          tc::tmem_wait_ld();
+          float sm[32];
+          uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) sm[j] = 0.f;
-      for (int tl = 0; tl < ri.ntiles; ++tl) {
-        uint32_t r[32];
-        tc::tmem_ld32(tbase + lane_off + tl * PH + hh * 32, r);
-        tc::tmem_wait_ld();
-        const int u = tl * PT + sq * 32 + lane;
-        const bool valid = u < ri.n_items;
-        const float sc = valid ? isc[u] : 0.f;
-        const float f = sc * ri.qscale;
-        uint32_t pw[16];
+          for (int j = 0; j < 32; j += 2) {
+            const float2 mm = *reinterpret_cast<const float2 *>(Ms + hh * 32 + j);
+            const float da = valid ? __uint_as_float(r[j]) * f - mm.x : -INFINITY;
+            const float db = valid ? __uint_as_float(r[j + 1]) * f - mm.y : -INFINITY;
+            over |= (da > thr) | (db > thr);
+            const float pa = ex2(da), pb = ex2(db);
+            sm[j] = pa;
+            sm[j + 1] = pb;
+            const __half2 v = __floats2half2_rn(pa * sc, pb * sc);
+            pk[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+          }
+          const int ul = sq * 32 + lane;
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 mm = *reinterpret_cast<const float2 *>(Ms + hh * 32 + j);
-          const float pa = valid ? ex2(__uint_as_float(r[j]) * f - mm.x) : 0.f;
-          const float pb = valid ? ex2(__uint_as_float(r[j + 1]) * f - mm.y) : 0.f;
-          sm[j] += pa;
-          sm[j + 1] += pb;
-          const __half2 v = __floats2half2_rn(pa * sc, pb * sc);
-          pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+          for (int hg = 0; hg < 4; ++hg)
+            *reinterpret_cast<uint4 *>(smem + S_PT + ppt_off(ul, hh * 4 + hg)) =
+                make_uint4(pk[4 * hg], pk[4 * hg + 1], pk[4 * hg + 2], pk[4 * hg + 3]);
+          reds[sq * PH + hh * 32 + lane] = warp_transpose_reduce<false>(sm);
         }
-#pragma unroll
-        for (int hg = 0; hg < 4; ++hg)
-          *reinterpret_cast<uint4 *>(smem + S_PT + ppt_off(u, hh * 4 + hg)) =
-              make_uint4(pw[4 * hg], pw[4 * hg + 1], pw[4 * hg + 2], pw[4 * hg + 3]);
+        if (detect && over) slow[ntile & 1] = 1;
+      };
+
+      bool need_max = tl == 0;
+      if (!need_max) {
+        p_phase(true);
+        named_sync(2, kSoft);
+        need_max = slow[ntile & 1] != 0;
+        // the next tile's flags (last read before this barrier) start clear
+        if (stid == 0) { slow[(ntile + 1) & 1] = 0; flag[(ntile + 1) & 1] = 0; }
       }
-      red[sq * PH + hh * 32 + lane] = warp_transpose_reduce<false>(sm);
+      if (need_max) {
+        // tile maximum of x = score * scale * log2(e), per head
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r[32];
+          tc::tmem_ld32(tbase + lane_off + kSCol + hh * 32, r);
+          tc::tmem_wait_ld();
+          float mx[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mx[j] = valid ? __uint_as_float(r[j]) * f : -INFINITY;
+          redm[sq * PH + hh * 32 + lane] = warp_transpose_reduce<true>(mx);
+        }
+        named_sync(2, kSoft);
+        if (stid == 0) { slow[(ntile + 1) & 1] = 0; flag[(ntile + 1) & 1] = 0; }
+        if (stid < PH) {
+          const float mt = fmaxf(fmaxf(redm[stid], redm[PH + stid]), fmaxf(redm[2 * PH + stid], redm[3 * PH + stid]));
+          const float mo = Mh[stid];
+          float fc = 1.f;
+          if (mt > mo + kPRescaleLog2) {
+            fc = mo == -INFINITY ? 0.f : ex2(mo - mt);
+            Lh[stid] *= fc;
+            Mh[stid] = mt;
+            if (tl > 0) flag[ntile & 1] = 1;
+          }
+          fac[stid] = fc;
+          Ms[stid] = Mh[stid] + ri.eshift;
+        }
+        named_sync(2, kSoft);
+        if (flag[ntile & 1]) {
+          // O^T holds the row's earlier tiles (their MMAs completed before this
+          // tile's scores): scale head column h of every d block by fac[h]
+#pragma unroll 1
+          for (int c = 0; c < kNdb * 2; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld32(tbase + lane_off + kOCol + c * 32, o);
+            tc::tmem_wait_ld();
+            const float *fcp = fac + (c & 1) * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * fcp[j]);
+            tc::tmem_st32(tbase + lane_off + kOCol + c * 32, o);
+          }
+          tc::tmem_wait_st();
+        }
+        p_phase(false);
+      }
+      tc::fence_proxy_async_smem();
+      tc::fence_before_sync();
+      named_sync(2, kSoft);
+      if (stid == 0) {
+        tc::mbar_arrive(&bars[B_PFULL]);
+        // the row's scales are no longer read
+        if (tl == ri.ntiles - 1) tc::mbar_arrive(&bars[B_FREE + par]);
+      }
+      if (stid < PH) Lh[stid] += (reds[stid] + reds[PH + stid]) + (reds[2 * PH + stid] + reds[3 * PH + stid]);
     }
-    tc::fence_proxy_async_smem();
-    tc::fence_before_sync();
+
+    // epilogue: O^T block dblk, lanes = d, columns = heads
+    pwait(&bars[B_OFULL], it & 1, misc, a.status);
+    tc::fence_after_sync();
     named_sync(2, kSoft);
-    if (stid == 0) tc::mbar_arrive(&bars[B_PTFULL]);
     if (stid < PH) {
-      const float L = red[stid] + red[PH + stid] + red[2 * PH + stid] + red[3 * PH + stid];
-      Lh[stid] = L;
+      const float L = Lh[stid];
       invL[stid] = 1.f / L;
       if (a.lse) a.lse[(int64_t)ri.row * PH + stid] = (Mh[stid] + ri.eshift + log2f(L)) * 0.6931471805599453f;
     }
     named_sync(2, kSoft);
-
-    // epilogue: O^T block dblk, lanes = d, columns = heads
     __nv_bfloat16 *orow = a.out + (int64_t)ri.row * PH * PD;
 #pragma unroll 1
-    for (int dblk = 0; dblk < PD / PDB; ++dblk) {
-      const uint32_t ob = ouse & 1u, use = ouse >> 1;
-      pwait(&bars[B_OFULL + ob], use & 1u, misc, a.status);
-      tc::fence_after_sync();
+    for (int dblk = 0; dblk < kNdb; ++dblk) {
       uint32_t r0[32], r1[32];
-      tc::tmem_ld32(tbase + lane_off + kOCol + ob * PH, r0);
-      tc::tmem_ld32(tbase + lane_off + kOCol + ob * PH + 32, r1);
+      tc::tmem_ld32(tbase + lane_off + kOCol + dblk * PH, r0);
+      tc::tmem_ld32(tbase + lane_off + kOCol + dblk * PH + 32, r1);
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&bars[B_OEMPTY + ob]);
-      ++ouse;
+      if (dblk == kNdb - 1) {
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars[B_OEMPTY]);
+      }
       __nv_bfloat16 *o = orow + dblk * PDB + sq * 32 + lane;
 #pragma unroll
       for (int j = 0; j < 32; ++j) o[j * PD] = __float2bfloat16_rn(__uint_as_float(r0[j]) * invL[j]);
 #pragma unroll
       for (int j = 0; j < 32; ++j) o[(32 + j) * PD] = __float2bfloat16_rn(__uint_as_float(r1[j]) * invL[32 + j]);
     }
+    // invL, Mh and Lh are reset or rewritten only after every thread is done
+    named_sync(2, kSoft);
   }
 }
 
@@ -520,66 +626,57 @@ __device__ __forceinline__ void run_mma(const PArgs &a, unsigned char *smem, int
   const uint32_t sbase = tc::smem_u32(smem);
   const uint32_t idesc_qk = tc::idesc_f16_f32(128, PH, 0, 0);
   const uint32_t idesc_pv = tc::idesc_f16_f32(128, PH, 1, 1);
-  uint32_t ncons = 0, ouse = 0;
+  uint32_t ntile = 0;
 
   for (int it = 0; it < nrows; ++it) {
     const int par = it & 1;
     pwait(&bars[B_READY + par], (it >> 1) & 1, misc, a.status);
     const int ntiles = info[par].ntiles;
-    // pass 1: S^T[tile] += K[tile, dblk] . Q[:, dblk]^T
-    for (int j = 0; j < ntiles * (PD / PDB); ++j) {
-      const uint32_t slot = ncons & 1u, use = ncons >> 1;
-      pwait(&bars[B_FULL + slot], use & 1u, misc, a.status);
-      tc::fence_after_sync();
-      if (leader) {
-        const int tile = j >> 2, dblk = j & 3;
-        const uint32_t kvb = sbase + S_KV + slot * KV_BYTES;
-#pragma unroll
-        for (int k = 0; k < PDB / 16; ++k) {
-          // A = K tile (M = items, K = d), K-major: LBO = d-group step, SBO = item-group step
-          const uint64_t ad = tc::smem_desc(kvb + k * 4096, 2048, 128);
-          // B = Q (N = heads, K = d), K-major: LBO = d-group step, SBO = head-group step
-          const uint64_t bd = tc::smem_desc(sbase + S_Q + (dblk * 16 + 2 * k) * 1024, 1024, 128);
-          tc::mma_bf16_ss(tbase + tile * PH, ad, bd, idesc_qk, (dblk > 0 || k > 0));
-        }
-        tc::mma_commit(&bars[B_EMPTY + slot]);
-      }
-      __syncwarp();
-      ++ncons;
-    }
-    if (leader) tc::mma_commit(&bars[B_P1DONE]);
-    __syncwarp();
-    pwait(&bars[B_PTFULL], it & 1, misc, a.status);
-    tc::fence_after_sync();
-    // pass 2: O^T[dblk] = sum over tiles of V^T[tile, dblk] . P^T[tile]
-    for (int dblk = 0; dblk < PD / PDB; ++dblk) {
-      const uint32_t ob = ouse & 1u, ou = ouse >> 1;
-      if (ou > 0) pwait(&bars[B_OEMPTY + ob], (ou - 1) & 1u, misc, a.status);
-      tc::fence_after_sync();
-      for (int tile = 0; tile < ntiles; ++tile) {
-        const uint32_t slot = ncons & 1u, use = ncons >> 1;
-        pwait(&bars[B_FULL + slot], use & 1u, misc, a.status);
+    for (int tl = 0; tl < ntiles; ++tl, ++ntile) {
+      // S^T = K_tile . Q^T, one d block per ring slot
+      for (int dblk = 0; dblk < kNdb; ++dblk) {
+        pwait(&bars[B_FULL + dblk], ntile & 1, misc, a.status);
         tc::fence_after_sync();
         if (leader) {
-          const uint32_t kvb = sbase + S_KV + slot * KV_BYTES;
+          const uint32_t kvb = sbase + S_KV + dblk * KV_BYTES;
+#pragma unroll
+          for (int k = 0; k < PDB / 16; ++k) {
+            // A = K tile (M = items, K = d), K-major: LBO = d-group step, SBO = item-group step
+            const uint64_t ad = tc::smem_desc(kvb + k * 4096, 2048, 128);
+            // B = Q (N = heads, K = d), K-major: LBO = d-group step, SBO = head-group step
+            const uint64_t bd = tc::smem_desc(sbase + S_Q + (dblk * 16 + 2 * k) * 1024, 1024, 128);
+            tc::mma_bf16_ss(tbase + kSCol, ad, bd, idesc_qk, (dblk > 0 || k > 0));
+          }
+        }
+        __syncwarp();
+      }
+      if (leader) {
+        tc::mma_commit(&bars[B_SFULL]);
+        if (tl == ntiles - 1) tc::mma_commit(&bars[B_QFREE]);
+      }
+      __syncwarp();
+      // the previous row's epilogue has read O^T before its first tile overwrites it
+      if (tl == 0 && it > 0) pwait(&bars[B_OEMPTY], (it - 1) & 1, misc, a.status);
+      pwait(&bars[B_PFULL], ntile & 1, misc, a.status);
+      tc::fence_after_sync();
+      // O^T[dblk] += V^T_tile[dblk] . P^T; the slot is free after these MMAs
+      if (leader) {
+        for (int dblk = 0; dblk < kNdb; ++dblk) {
+          const uint32_t kvb = sbase + S_KV + dblk * KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < PT / 16; ++kk) {
             // A = V^T (M = d, K = items), MN-major: LBO = item-group step, SBO = d-group step
             const uint64_t ad = tc::smem_desc(kvb + kk * 256, 128, 2048);
             // B = P^T (N = heads, K = items), MN-major: LBO = item-group step, SBO = head-group step
-            const uint64_t bd = tc::smem_desc(sbase + S_PT + (tile * 16 + 2 * kk) * 1024, 1024, 128);
-            tc::mma_bf16_ss(tbase + kOCol + ob * PH, ad, bd, idesc_pv, (tile > 0 || kk > 0));
+            const uint64_t bd = tc::smem_desc(sbase + S_PT + (2 * kk) * 1024, 1024, 128);
+            tc::mma_bf16_ss(tbase + kOCol + dblk * PH, ad, bd, idesc_pv, (tl > 0 || kk > 0));
           }
-          tc::mma_commit(&bars[B_EMPTY + slot]);
+          tc::mma_commit(&bars[B_EMPTY + dblk]);
         }
-        __syncwarp();
-        ++ncons;
       }
-      if (leader) tc::mma_commit(&bars[B_OFULL + ob]);
       __syncwarp();
-      ++ouse;
     }
-    if (leader) tc::mma_commit(&bars[B_P2DONE]);
+    if (leader) tc::mma_commit(&bars[B_OFULL]);
     __syncwarp();
   }
   // every MMA issued above completes before the TMEM is released
@@ -598,22 +695,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_kernel(const PArgs
   const int tid = threadIdx.x, warp = tid >> 5;
   if (tid == 0) {
     misc->abort = 0;
-    tc::mbar_init(&bars[B_FULL + 0], kProd / 32);
-    tc::mbar_init(&bars[B_FULL + 1], kProd / 32);
-    tc::mbar_init(&bars[B_EMPTY + 0], 1);
-    tc::mbar_init(&bars[B_EMPTY + 1], 1);
-    tc::mbar_init(&bars[B_READY + 0], kProd / 32);
-    tc::mbar_init(&bars[B_READY + 1], kProd / 32);
-    tc::mbar_init(&bars[B_P1DONE], 1);
-    tc::mbar_init(&bars[B_PTFULL], 1);
-    tc::mbar_init(&bars[B_P2DONE], 1);
-    tc::mbar_init(&bars[B_OFULL + 0], 1);
-    tc::mbar_init(&bars[B_OFULL + 1], 1);
-    tc::mbar_init(&bars[B_OEMPTY + 0], kSoft / 32);
-    tc::mbar_init(&bars[B_OEMPTY + 1], kSoft / 32);
+    for (int s = 0; s < kNdb; ++s) {
+      tc::mbar_init(&bars[B_FULL + s], kProd / 32);
+      tc::mbar_init(&bars[B_EMPTY + s], 1);
+    }
+    for (int p = 0; p < 2; ++p) {
+      tc::mbar_init(&bars[B_READY + p], kSetup / 32);
+      tc::mbar_init(&bars[B_ITEMS + p], kSetup / 32);
+      tc::mbar_init(&bars[B_FREE + p], kProd / 32 + 1);
+    }
+    tc::mbar_init(&bars[B_QFREE], 1);
+    tc::mbar_init(&bars[B_SFULL], 1);
+    tc::mbar_init(&bars[B_PFULL], 1);
+    tc::mbar_init(&bars[B_OFULL], 1);
+    tc::mbar_init(&bars[B_OEMPTY], kSoft / 32);
     tc::mbar_init(&bars[B_FINAL], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (tid < 4) reinterpret_cast<int *>(smem + S_FLAG)[tid] = 0;
   if (warp == 0) tc::tmem_alloc(&misc->tmem_base, 512);
   tc::fence_before_sync();
   __syncthreads();
@@ -623,7 +722,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_prefill_kernel(const PArgs
 
   if (warp < kProd / 32) run_producers(a, smem, nrows);
   else if (warp < kMmaWarp) run_softmax(a, smem, nrows, tbase);
-  else run_mma(a, smem, nrows, tbase);
+  else if (warp == kMmaWarp) run_mma(a, smem, nrows, tbase);
+  else run_setup(a, smem, nrows);
 
   tc::fence_before_sync();
   __syncthreads();
