@@ -168,17 +168,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Two E4M3 codes -> two fp16 (exact: every finite E4M3 value is an fp16).
-__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four E4M3 codes (byte i of w is code i) -> four fp16, codes 0-1 in `lo`
+// and 2-3 in `hi`, the lower code in the lower half (exact: every finite
+// E4M3 value is an fp16).  One PTX cvt per pair of codes.
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
+// 16 E4M3 codes -> 16 fp16, codes 0-7 in `lo` and 8-15 in `hi`
 __device__ __forceinline__ void cvt16(const uint4 &c, uint4 &lo, uint4 &hi) {
-  lo = make_uint4(e4m3x2_to_h2(c.x & 0xFFFFu), e4m3x2_to_h2(c.x >> 16), e4m3x2_to_h2(c.y & 0xFFFFu),
-                  e4m3x2_to_h2(c.y >> 16));
-  hi = make_uint4(e4m3x2_to_h2(c.z & 0xFFFFu), e4m3x2_to_h2(c.z >> 16), e4m3x2_to_h2(c.w & 0xFFFFu),
-                  e4m3x2_to_h2(c.w >> 16));
+  e4m3x4_to_h2x2(c.x, lo.x, lo.y);
+  e4m3x4_to_h2x2(c.y, lo.z, lo.w);
+  e4m3x4_to_h2x2(c.z, hi.x, hi.y);
+  e4m3x4_to_h2x2(c.w, hi.z, hi.w);
 }
 
 // Two bf16 (packed) times an exact power of two -> two fp16 (packed).
@@ -313,7 +318,7 @@ __device__ __forceinline__ void run_setup(const PArgs &a, unsigned char *smem, i
     // Q row max (thread st holds head st) and the largest scale
     const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + (int64_t)row * PH * PD) + st * (PD / 8);
     uint32_t mq = 0;
-#pragma unroll 8
+#pragma unroll 16
     for (int k = 0; k < PD / 8; ++k) {
       const uint4 v = __ldg(qg + k);
       mq = __vmaxu2(mq, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
@@ -340,14 +345,27 @@ __device__ __forceinline__ void run_setup(const PArgs &a, unsigned char *smem, i
       ri.eshift = (float)min(112, max(-110, e - 133));
       ri.pad1[0] = ri.pad1[1] = 0.f;
     }
-    // Q in fp16: the buffer is free once the previous row's last scores are complete
-    if (it > 0) pwait(&bars[B_QFREE], (it - 1) & 1, misc, a.status);
+    // Q in fp16, 16 chunks of 8 per batch (the first batch is loaded before
+    // the wait): the buffer is free once the previous row's last scores are
+    // complete
     unsigned char *qs_ = smem + S_Q;
-#pragma unroll 8
-    for (int k = 0; k < PD / 8; ++k) {
-      const uint4 v = __ldg(qg + k);
-      *reinterpret_cast<uint4 *>(qs_ + pq_off(st, k)) =
-          make_uint4(bf2_to_h2(v.x, fq), bf2_to_h2(v.y, fq), bf2_to_h2(v.z, fq), bf2_to_h2(v.w, fq));
+    constexpr int kQb = 16;
+    uint4 qv[kQb];
+#pragma unroll
+    for (int k = 0; k < kQb; ++k) qv[k] = __ldg(qg + k);
+    if (it > 0) pwait(&bars[B_QFREE], (it - 1) & 1, misc, a.status);
+#pragma unroll 1
+    for (int k0 = 0; k0 < PD / 8; k0 += kQb) {
+#pragma unroll
+      for (int k = 0; k < kQb; ++k) {
+        const uint4 v = qv[k];
+        *reinterpret_cast<uint4 *>(qs_ + pq_off(st, k0 + k)) =
+            make_uint4(bf2_to_h2(v.x, fq), bf2_to_h2(v.y, fq), bf2_to_h2(v.z, fq), bf2_to_h2(v.w, fq));
+      }
+      if (k0 + kQb < PD / 8) {
+#pragma unroll
+        for (int k = 0; k < kQb; ++k) qv[k] = __ldg(qg + k0 + kQb + k);
+      }
     }
     tc::fence_proxy_async_smem();
     // pred is reused by the next row
