@@ -548,7 +548,7 @@ def roofline(name, work, ms, peaks, src, wl):
 
 def kernel_traffic(call, workload):
     """DRAM bytes per launch of a call from the committed ncu summary, or None
-    when absent or when the kernel sources changed since it was taken."""
+    when absent or when the kernel's sources changed since it was taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -557,15 +557,29 @@ def kernel_traffic(call, workload):
     rec = d.get(workload, {}).get(call)
     if not rec:
         return None
-    if rec.get("source_sha") != source_sha():
+    if rec.get("source_sha") != source_sha(rec.get("kernel", "")):
         return None
     return rec.get("dram_bytes")
 
 
-def source_sha():
-    h = hashlib.sha256()
+# the source files each profiled kernel is built from (its own file and the
+# shared device headers)
+KERNEL_SOURCES = {
+    "attend_tc_kernel": ["attend_tc.cu"],
+    "attend_prefill_kernel": ["attend_prefill.cu"],
+    "index_decode_kernel<4>": ["indexer.cu"],
+}
+SHARED_SOURCES = ["common.cuh", "tc.cuh"]
+
+
+def source_sha(kernel):
+    """Hash of the sources a kernel is built from; unknown kernels hash every
+    file of the CUDA sources."""
     csrc = os.path.join(ROOT, "compressed_sparse_attention_16_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    files = KERNEL_SOURCES.get(kernel)
+    files = sorted(files + SHARED_SOURCES) if files else sorted(os.listdir(csrc))
+    h = hashlib.sha256()
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
