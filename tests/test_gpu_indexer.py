@@ -160,3 +160,27 @@ def test_prefill_path_random_two_sequences():
     _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
     inp2 = synth.indexer_inputs(B, Tq, N, 2, 64, seed=14)
     _compare(inp2.qI, inp2.w, inp2.kI, pos, m, 64, N)
+
+
+def test_scan_collect_path():
+    """64 decode rows over 20,000 entries: more than one CTA per SM pair can
+    hold (8,192 entries each), so the two-kernel tensor-core path (per-slice
+    scores and histograms, then the threshold and collection) runs."""
+    B, Tq, N, m, K = 1, 64, 20000, 4, 512
+    inp = synth.indexer_inputs(B, Tq, N, 4, 64, seed=21)
+    g = torch.Generator().manual_seed(21)
+    pos = torch.randint(0, 4 * N + 10, (B, Tq), generator=g, dtype=torch.int32)
+    pos[0, :6] = torch.tensor([0, 4 * 512 - 1, 4 * 512, 4 * N - 1, 4 * N + 9, 4 * 5000], dtype=torch.int32)
+    _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
+
+
+@pytest.mark.parametrize("HI,dI", [(8, 32), (2, 32)])
+def test_split_merge_path(HI, dI):
+    """Few rows over >= 2,048 entries with an indexer shape the tensor-core
+    paths do not take: per-slice candidates, then a merge per row."""
+    B, Tq, N, m, K = 1, 16, 5000, 4, 512
+    inp = synth.indexer_inputs(B, Tq, N, HI, dI, seed=22 + HI)
+    g = torch.Generator().manual_seed(22)
+    pos = torch.randint(0, 4 * N + 10, (B, Tq), generator=g, dtype=torch.int32)
+    pos[0, :4] = torch.tensor([1, 4 * 512 - 1, 4 * 512 + 3, 4 * N - 1], dtype=torch.int32)
+    _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
