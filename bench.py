@@ -771,6 +771,16 @@ def kernel_case(args, wl):
         codes = torch.empty((B, max(1, n_tok // m), D), dtype=torch.uint8, device=dev)
         scales = torch.empty((B, max(1, n_tok // m)), device=dev)
         fn = lambda: csa.compress(x, z, m, codes, scales)
+    elif case == "quantize_mxfp4":
+        # fp32 indexer queries of the workload (B * Tq * HI rows of dI values) to MXFP4
+        rows = B * Tq * max(wl.HI, 1)
+        cols = max(wl.dI, 32)
+        g = torch.Generator(device=dev).manual_seed(0)
+        xq = torch.randn((rows, cols), generator=g, device=dev)
+        qcodes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+        qscales = torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+        case_bytes = rows * cols * 4 + rows * cols // 2 + rows * cols // 32
+        fn = lambda: csa.quantize_mxfp4(xq, qcodes, qscales)
     else:
         raise SystemExit(f"unknown kernel case {case}")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -790,9 +800,15 @@ def kernel_case(args, wl):
     torch.cuda.synchronize()
     csa.sync_status()
     ms = [a.elapsed_time(b) for a, b in times]
-    print(json.dumps({"kernel_case": case, "workload": wl.name, "ms_mean": float(np.mean(ms)),
-                      "ms_min": float(np.min(ms)), "calls": args.steps,
-                      "device_bytes": int(torch.cuda.max_memory_allocated(dev))}))
+    line = {"kernel_case": case, "workload": wl.name, "ms_mean": float(np.mean(ms)),
+            "ms_min": float(np.min(ms)), "calls": args.steps,
+            "device_bytes": int(torch.cuda.max_memory_allocated(dev))}
+    if case == "quantize_mxfp4":
+        peaks, src = load_peaks()
+        gbs = case_bytes / (float(np.mean(ms)) / 1e3) / 1e9
+        line.update({"algorithmic_bytes": int(case_bytes), "achieved_gbs": gbs,
+                     "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak_source": src})
+    print(json.dumps(line))
 
 
 def main():
@@ -807,7 +823,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
     ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
-                    help="run one library call (index_topk, attend, hca_attend, compress_entry) alone on "
+                    help="run one library call (index_topk, attend, hca_attend, compress_entry, "
+                         "quantize_mxfp4) alone on "
                          "inputs of the workload's shape; for profilers")
     args = ap.parse_args()
     import synth

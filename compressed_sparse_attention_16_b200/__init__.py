@@ -38,6 +38,7 @@ SYMBOLS = (
     "csa_sync_status",
     "csa_version",
     "csa_launch_count",
+    "csa_quantize_mxfp4",
     "csa_selftest_timeout",
 )
 
@@ -107,6 +108,8 @@ def lib() -> ctypes.CDLL:
     L.csa_launch_count.restype = ctypes.c_uint64
     L.csa_selftest_timeout.argtypes = [ctypes.c_uint64, _P]
     L.csa_selftest_timeout.restype = ctypes.c_int
+    L.csa_quantize_mxfp4.argtypes = [_P, _I64, _I32, _P, _P, _P]
+    L.csa_quantize_mxfp4.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -166,6 +169,19 @@ def compress(x: torch.Tensor, z: torch.Tensor, m: int, codes: torch.Tensor, scal
                               _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
                               dst_first, codes.shape[1], ring_cap,
                               _ptr(pooled, torch.float32, "pooled", dev), _stream(stream)))
+
+
+def quantize_mxfp4(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    """csa_quantize_mxfp4: fp32 x [rows, cols] (cols a multiple of 32) to packed
+    E2M1 codes u8 [rows, cols/2] and E8M0 block scales u8 [rows, cols/32]."""
+    if x.dim() != 2:
+        raise ValueError("x must be [rows, cols]")
+    rows, cols = x.shape
+    if codes.shape != (rows, cols // 2) or scales.shape != (rows, cols // 32):
+        raise ValueError("codes must be [rows, cols/2] and scales [rows, cols/32]")
+    dev = x.device
+    _check(lib().csa_quantize_mxfp4(_ptr(x, torch.float32, "x"), rows, cols, _ptr(codes, torch.uint8, "codes", dev),
+                                    _ptr(scales, torch.uint8, "scales", dev), _stream(stream)))
 
 
 def index_topk_workspace(dims: Dims) -> int:

@@ -213,6 +213,30 @@ int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
 const char *csa_last_error(void);
 
 /*
+ * csa_quantize_mxfp4 -- fp32 values to MXFP4 (E2M1 elements, one E8M0 scale
+ * per 32 consecutive elements), the format the indexer consumes.
+ * ("DeepSeek V4 Flash：知っておくべき284Bパラメータのオープンソースモデル"
+ *  (studioglobal.ai), "FP4/FP8混合精度": FP4 values are MXFP4, two per byte;
+ *  jiwasawa.github.io DeepSeek-V4 article, "限界を押し広げるインフラストラクチャ
+ *  の最適化": FP4 on the indexer's QK path.)
+ *
+ * For every block of 32 consecutive elements v of a row:
+ *     X     = max(floor(log2(max |v|)) - 2, -127)   (-127 for an all-zero block)
+ *     scale = E8M0 code X + 127                     (the value 2^X)
+ *     code  = E2M1(v / 2^X), round-to-nearest-even, saturating at +-6; the
+ *             sign is kept (a negative value that rounds to zero is -0, 0x8)
+ * v / 2^X is exact in fp32, so every code and scale is fully determined.
+ *
+ *   x        fp32 [rows, cols], finite values
+ *   codes    u8   [rows, cols/2]   packed E2M1, the even element in the low nibble
+ *   scales   u8   [rows, cols/32]  E8M0 codes
+ * Requires cols a positive multiple of 32, rows >= 0 (0 is a no-op); x
+ * 16-byte and codes 4-byte aligned.  CSA_ERR_INVALID for anything else.
+ */
+int csa_quantize_mxfp4(const float *x, int64_t rows, int32_t cols, uint8_t *codes, uint8_t *scales,
+                       csa_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device status word,
  * which kernels set when a bounded device-side wait gives up.  Returns CSA_OK,
  * CSA_ERR_TIMEOUT, or CSA_ERR_CUDA if the stream itself reported an error.

@@ -121,6 +121,82 @@ def e2m1_unpack(packed) -> np.ndarray:
     return out
 
 
+# E2M1 magnitudes in code order (codes 0..7; bit 3 is the sign)
+E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def e2m1_encode(values) -> np.ndarray:
+    """Round exactly-known values (float64) to E2M1 codes (0..15).
+
+    Nearest value of the grid, ties to the code with an even mantissa bit
+    (the even code), magnitudes above 6 saturate to 6.  The sign is kept,
+    so a negative value that rounds to zero gives the code of -0 (0x8).
+    """
+    v = np.asarray(values, dtype=np.float64)
+    if np.isnan(v).any():
+        raise ValueError("e2m1_encode: NaN")
+    mag = np.minimum(np.abs(v), 6.0)
+    grid = np.asarray(E2M1_GRID)
+    lo = np.clip(np.searchsorted(grid, mag, side="right") - 1, 0, 7)   # grid[lo] <= mag
+    hi = np.minimum(lo + 1, 7)
+    d_lo = mag - grid[lo]
+    d_hi = grid[hi] - mag
+    up = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0) & (hi != lo))
+    code = np.where(up, hi, lo).astype(np.uint8)
+    sign = np.where(np.signbit(v), 0x8, 0x0).astype(np.uint8)
+    return (code | sign).astype(np.uint8)
+
+
+def e2m1_pack(codes) -> np.ndarray:
+    """Pack codes [..., d] (d even) two per byte: element 2j in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+# --------------------------------------------------------------------------
+# E8M0: an 8-bit power-of-two scale, 2**(code - 127); 0xFF is NaN.
+# --------------------------------------------------------------------------
+
+
+def e8m0_decode(codes) -> np.ndarray:
+    c = np.asarray(codes).astype(np.int64)
+    return np.where(c == 0xFF, np.nan, np.exp2((c - 127).astype(np.float64)))
+
+
+# --------------------------------------------------------------------------
+# MXFP4: blocks of 32 elements, E2M1 elements and one E8M0 scale per block.
+# --------------------------------------------------------------------------
+MX_BLOCK = 32
+
+
+def mxfp4_quantize(x):
+    """Quantise fp32 values [rows, cols] (cols a multiple of 32) to MXFP4.
+
+    Source: "DeepSeek V4 Flash：知っておくべき284Bパラメータのオープンソースモデル"
+    (studioglobal.ai), section "FP4/FP8混合精度" -- FP4 values are MXFP4,
+    packed two per byte.  The pages give no rounding rule; this is the OCP
+    microscaling conversion written out: per block of 32 consecutive
+    elements, X = floor(log2(max|v|)) - 2 (2 being the exponent of the
+    largest E2M1 value, 6 = 1.5 * 2**2), at least -127 (an all-zero block
+    takes -127); scale = 2**X stored as the E8M0 code X + 127; each element
+    v / 2**X (exact) rounded by e2m1_encode.
+
+    Returns (packed codes u8 [rows, cols/2], scale codes u8 [rows, cols/32]).
+    """
+    v = np.asarray(x, dtype=np.float32).astype(np.float64)
+    if v.ndim != 2 or v.shape[1] % MX_BLOCK:
+        raise ValueError("mxfp4_quantize: expects [rows, cols] with cols a multiple of 32")
+    rows, cols = v.shape
+    blocks = v.reshape(rows, cols // MX_BLOCK, MX_BLOCK)
+    amax = np.abs(blocks).max(axis=-1)
+    _, e = np.frexp(amax)                      # amax = f * 2**e, f in [0.5, 1): floor(log2) = e - 1
+    X = np.where(amax > 0, e - 1 - 2, -127)
+    X = np.maximum(X, -127).astype(np.int64)
+    r = blocks / np.exp2(X.astype(np.float64))[..., None]
+    codes = e2m1_encode(r).reshape(rows, cols)
+    return e2m1_pack(codes), (X + 127).astype(np.uint8)
+
+
 # --------------------------------------------------------------------------
 # bf16: the top half of an IEEE binary32.
 # --------------------------------------------------------------------------

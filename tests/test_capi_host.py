@@ -120,3 +120,20 @@ def test_binding_requires_cuda_tensors():
     x = torch.zeros(1, 8, 64)
     with pytest.raises(ValueError):
         csa.compress(x, x, 4, torch.zeros(1, 2, 64, dtype=torch.uint8), torch.zeros(1, 2))
+
+
+def test_quantize_mxfp4_rejects_bad_arguments():
+    L = csa.lib()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    rc, msg = _rc(L.csa_quantize_mxfp4, fake, 4, 48, fake, fake, None)
+    assert rc == csa.CSA_ERR_INVALID and "multiple of 32" in msg
+    rc, _ = _rc(L.csa_quantize_mxfp4, fake, -1, 64, fake, fake, None)
+    assert rc == csa.CSA_ERR_INVALID
+    rc, msg = _rc(L.csa_quantize_mxfp4, None, 4, 64, fake, fake, None)
+    assert rc == csa.CSA_ERR_INVALID and "NULL" in msg
+    rc, msg = _rc(L.csa_quantize_mxfp4, ctypes.c_void_p((1 << 20) + 8), 4, 64, fake, fake, None)
+    assert rc == csa.CSA_ERR_INVALID and "misaligned" in msg
+    rc, msg = _rc(L.csa_quantize_mxfp4, fake, 4, 64, ctypes.c_void_p((1 << 20) + 2), fake, None)
+    assert rc == csa.CSA_ERR_INVALID and "misaligned" in msg
+    # no rows is a no-op that succeeds without a device
+    assert L.csa_quantize_mxfp4(fake, 0, 64, fake, fake, None) == 0

@@ -5,7 +5,8 @@ import ml_dtypes
 import numpy as np
 import pytest
 
-from oracle.formats import bf16_decode, e2m1_decode, e2m1_unpack, e4m3_decode, e4m3_encode
+from oracle.formats import (E2M1_GRID, bf16_decode, e2m1_decode, e2m1_encode, e2m1_pack, e2m1_unpack, e4m3_decode,
+                            e4m3_encode, e8m0_decode, mxfp4_quantize)
 
 ALL = np.arange(256, dtype=np.uint8)
 
@@ -100,3 +101,84 @@ def test_bf16_decode_matches_ml_dtypes():
     ok = ~np.isnan(ref)
     assert np.array_equal(np.isnan(ref), np.isnan(got))
     assert np.array_equal(ref[ok], got[ok])
+
+
+# ---------------------------------------------------------------- E2M1 encode, E8M0, MXFP4
+
+
+def _e2m1_grid_inputs():
+    """Every grid value, every midpoint (the ties), points one fp32 ulp either
+    side of each midpoint, values past 6, and the negatives of all of them."""
+    g = np.asarray(E2M1_GRID)
+    mids = (g[:-1] + g[1:]) / 2
+    pts = np.concatenate([g, mids, np.nextafter(mids.astype(np.float32), np.float32(0)).astype(np.float64),
+                          np.nextafter(mids.astype(np.float32), np.float32(9)).astype(np.float64),
+                          [6.5, 7.0, 7.999, 100.0, 1e-30, 0.1, 0.2499, 0.2501]])
+    rng = np.random.default_rng(5)
+    pts = np.concatenate([pts, rng.uniform(0, 7.99, 2000).astype(np.float32).astype(np.float64)])
+    return np.concatenate([pts, -pts])
+
+
+def test_e2m1_encode_matches_ml_dtypes():
+    v = _e2m1_grid_inputs()
+    ref = v.astype(np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    assert np.array_equal(e2m1_encode(v), ref)
+
+
+def test_e2m1_encode_is_nearest_even_bruteforce():
+    v = _e2m1_grid_inputs()
+    got = e2m1_encode(v)
+    dec = e2m1_decode(got)
+    grid = np.asarray(E2M1_GRID)
+    for x, c, d in zip(v, got, dec):
+        mag = min(abs(x), 6.0)
+        dist = np.abs(grid - mag)
+        best = np.flatnonzero(dist == dist.min())
+        k = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert abs(d) == grid[k] and (c & 0x8) == (0x8 if np.signbit(x) else 0)
+
+
+def test_e2m1_pack_inverts_unpack():
+    c = np.random.default_rng(6).integers(0, 16, (5, 64)).astype(np.uint8)
+    assert np.array_equal(e2m1_unpack(e2m1_pack(c)), c)
+
+
+def test_e8m0_decode_matches_ml_dtypes():
+    codes = np.arange(255, dtype=np.uint8)
+    ref = codes.view(ml_dtypes.float8_e8m0fnu).astype(np.float64)
+    assert np.array_equal(e8m0_decode(codes), ref)
+    assert np.isnan(e8m0_decode(np.array([255], dtype=np.uint8)))[0]
+
+
+def test_mxfp4_worked_block():
+    """One block worked by hand: max |v| = 13 -> floor(log2 13) = 3 -> X = 1
+    (scale code 128, 2^1); v / 2 = 3, -0.375, 0.125, 6.5, -0.25, 2.25, ...;
+    codes 3 -> 0b0101, -0.375 -> -0.5 (0b1001), 0.125 -> 0, 6.5 -> 6 (0b0111),
+    -0.25 -> -0 (tie to the even code, 0b1000), 2.25 -> 2 (0b0100)."""
+    v = np.zeros((1, 32), dtype=np.float32)
+    v[0, :6] = [6.0, -0.75, 0.25, 13.0, -0.5, 4.5]
+    codes, scales = mxfp4_quantize(v)
+    assert scales.tolist() == [[128]]
+    assert e2m1_unpack(codes)[0, :6].tolist() == [0x5, 0x9, 0x0, 0x7, 0x8, 0x4]
+    assert (e2m1_unpack(codes)[0, 6:] == 0).all()
+
+
+def test_mxfp4_scale_range_and_error_bound():
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((40, 128)) * np.exp2(rng.integers(-40, 40, (40, 1)))).astype(np.float32)
+    x[3, 32:64] = 0.0                      # an all-zero block
+    x[5, :32] = 1e-42                      # subnormal block
+    codes, scales = mxfp4_quantize(x)
+    X = scales.astype(np.int64) - 127
+    blocks = x.astype(np.float64).reshape(40, 4, 32)
+    amax = np.abs(blocks).max(-1)
+    normal = amax >= 2.0 ** -125
+    ratio = amax[normal] / np.exp2(X[normal])
+    assert ((ratio >= 4) & (ratio < 8)).all()
+    assert X[3, 1] == -127 and X[5, 0] == -127
+    dq = e2m1_decode(e2m1_unpack(codes)).reshape(40, 4, 32) * np.exp2(X)[..., None]
+    r = np.abs(blocks) / np.exp2(X)[..., None]
+    # half a grid step below 4 (at most 1 in the scaled units), saturation above 6
+    bound = np.where(r <= 6, np.where(r < 4, 0.5, 1.0), r - 6) * np.exp2(X)[..., None]
+    assert (np.abs(dq - blocks) <= bound + 1e-300).all()
+    assert (dq[3, 1] == 0).all()
