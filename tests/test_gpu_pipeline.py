@@ -185,3 +185,35 @@ def test_bounded_wait_expiry_is_reported_and_context_survives():
     scales = torch.empty((1, 2), device="cuda")
     csa.compress(x, torch.zeros_like(x), 4, codes, scales)
     csa.sync_status()
+
+
+def test_sharded_prefill_one_rank_equals_prefill():
+    """prefill_sharded on a one-rank NCCL group runs the same calls on the
+    same data as prefill: identical outputs (the multi-rank plumbing is
+    covered with gloo ranks on the CPU)."""
+    import socket
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    from compressed_sparse_attention_16_b200 import shard
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=timedelta(seconds=60))
+    try:
+        B, T, D, H, m, K, W = 1, 1030, 512, 64, 4, 64, 128
+        x, z = synth.tokens(B, T, D, 3)
+        q = synth.queries(B, T, H, D, 512 ** -0.5, 3)
+        ind = synth.indexer_inputs(B, T, T // m, 4, 64, 3)
+        x, z, q = x.cuda(), z.cuda(), q.cuda()
+        qI, w, kI = ind.qI.cuda(), ind.w.cuda(), ind.kI.cuda()
+        ref = pipeline.prefill(x, z, q, qI, w, kI, m=m, K=K, W=W)
+        got = shard.prefill_sharded(x, z, kI, q, qI, w, T=T, m=m, K=K, W=W)
+        torch.cuda.synchronize()
+        assert torch.equal(got.pos.cuda().long(), torch.arange(T, device="cuda"))
+        assert torch.equal(got.idx, ref.idx) and torch.equal(got.score, ref.score)
+        assert torch.equal(got.out, ref.out) and torch.equal(got.lse, ref.lse)
+    finally:
+        dist.destroy_process_group()
