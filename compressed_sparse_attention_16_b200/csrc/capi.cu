@@ -88,12 +88,17 @@ bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base
 }
 
 int set_smem_once(const void *kernel, int bytes, const char *name) {
+  // one slot per kernel instance that raises its limit: 27 in this library
+  // (the generic attention per D, the indexer paths per head count and
+  // indexer shape, the 128- and 64-head attention, the merge and the long
+  // pooling kernel), so 64 slots per device always suffice
+  constexpr int kSlots = 64;
   static std::mutex mu;
-  static const void *done[64][16] = {{nullptr}};
+  static const void *done[64][kSlots] = {{nullptr}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(CSA_ERR_CUDA, "%s: no device", name);
   std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < kSlots; ++i) {
     if (done[dev][i] == kernel) return CSA_OK;
     if (done[dev][i] == nullptr) {
       const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
