@@ -77,3 +77,24 @@ def test_traffic_follows_each_kernels_sources(tmp_path, monkeypatch):
         f.write("\n// edited\n")
     assert bench.kernel_traffic("index_topk", "wl") is None
 
+
+
+@pytest.mark.parametrize("name", ["tiny_prefill", "csa_decode_64k"])
+def test_reference_arm_line(name, monkeypatch):
+    """`bench.py --impl reference`: the oracle timed on the host cores, one
+    JSON line with the contract's keys (rank 0 only)."""
+    import types
+    monkeypatch.setenv("RANK", "0")
+    line = bench.reference_arm(types.SimpleNamespace(steps=1, warmup=0), synth.WORKLOADS[name])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == ("queries/s" if name == "tiny_prefill" else "tokens/s")
+    assert line["config"]["workload"] == name
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    json.dumps(line)
+    monkeypatch.setenv("RANK", "1")
+    assert bench.reference_arm(types.SimpleNamespace(steps=1, warmup=0), synth.WORKLOADS[name]) is None
