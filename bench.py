@@ -1,17 +1,21 @@
 #!/usr/bin/env python3
 """Benchmark of the hybrid compressed-attention path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl reference]
 
-Workloads (synthetic, seeded): csa_decode_64k (default), csa_decode_1m_incremental,
-hca_decode_1m, csa_prefill_128k, tiny_prefill.  A step is one pass of the whole path
-for one batch: decode -> append 4 tokens (pool one entry + 4 window tokens), indexer +
-top-k, attention; HCA decode -> append 128 tokens (one entry + window) then dense
-attention; prefill -> pool the whole sequence, index + select every position, attend.
+Workloads (synthetic, seeded): csa_decode_1m_incremental (the headline),
+csa_decode_64k, hca_decode_1m, csa_prefill_128k, tiny_prefill.  The default
+(`all`) times K steps of the headline, then up to 20 steps of every other
+workload, and prints the headline's figures at the top level of the line and
+every workload's under "workloads".  A step is one pass of the whole path for
+one batch: decode -> append 4 tokens (pool one entry + 4 window tokens), indexer
++ top-k, attention; HCA decode -> append 128 tokens (one entry + window) then
+dense attention; prefill -> pool the whole sequence, index + select every
+position, attend.
 
-Prints ONE JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
-independent sequences (weak scaling, no collective on the data path); times are the
-max over ranks.
+Prints ONE JSON line (rank 0).  With N > 1 every rank runs its own independent
+sequences (weak scaling, no collective on the data path); times are the max
+over ranks.  `--gpus N` without torchrun starts the N ranks itself.
 """
 from __future__ import annotations
 
@@ -369,10 +373,19 @@ def l2_flush(buf):
     buf.view(torch.int64).sum()
 
 
-def gpu_arm(args, wl):
+HEADLINE = "csa_decode_1m_incremental"
+# every configuration of the library's workload set, headline first
+ALL_WORKLOADS = (HEADLINE, "csa_decode_64k", "hca_decode_1m", "csa_prefill_128k", "tiny_prefill")
+# timed steps and CPU-baseline budget of the workloads after the headline
+SECONDARY_STEPS = 20
+SECONDARY_CPU_BUDGET_S = 6.0
+HBM_NOMINAL_GBS = 8000.0
+
+
+def init_ranks():
+    """(world, rank, local rank, device); joins the NCCL group when world > 1."""
     import torch
     import torch.distributed as dist
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -382,7 +395,15 @@ def gpu_arm(args, wl):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    peaks, peaks_src = load_peaks()
+    return world, rank, local, dev
+
+
+def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budget):
+    """Time `steps` steps of one workload on every rank; rank 0 gets the
+    workload's record (the other ranks None)."""
+    import torch
+    import torch.distributed as dist
+
     r = Runner(wl, seed=rank, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     use_graph = r.decode and not args.no_graph
@@ -399,7 +420,7 @@ def gpu_arm(args, wl):
         else:
             r.run(i)
     if use_graph:
-        for i in range(args.warmup, args.warmup + args.steps):
+        for i in range(args.warmup, args.warmup + steps):
             r.graph(i)
     barrier()
 
@@ -408,7 +429,7 @@ def gpu_arm(args, wl):
     step_events = []
     launches = 0
     wall0 = time.perf_counter()
-    for i in range(args.warmup, args.warmup + args.steps):
+    for i in range(args.warmup, args.warmup + steps):
         l2_flush(flush)                     # evict L2 between timed steps (outside the events)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -429,12 +450,12 @@ def gpu_arm(args, wl):
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
     step_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_events), world, dev)
-    ms_per_step = step_ms / args.steps
+    ms_per_step = step_ms / steps
     value = job_throughput(world, r.units_per_step, ms_per_step)
 
     # per-call device time: each call alone, cold L2, queued behind a bounded sleep
     per_call = {}
-    for i in range(args.warmup, args.warmup + min(args.steps, 5)):
+    for i in range(args.warmup, args.warmup + min(steps, 5)):
         for name, fn in r.calls(i):
             l2_flush(flush)
             torch.cuda._sleep(200000)
@@ -447,38 +468,93 @@ def gpu_arm(args, wl):
     torch.cuda.synchronize()
     call_ms = {k: float(np.mean([a.elapsed_time(b) for a, b in v])) for k, v in per_call.items()}
 
-    e2e = e2e_leg(r, args, world, dev, use_graph)
+    e2e = e2e_leg(r, args, world, dev, use_graph, steps)
+    r.graphs.clear()
+    del r, flush
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    work = op_work(wl)
+    dom = max(call_ms, key=lambda k: call_ms[k])
+    rec = {
+        "value": value, "unit": "queries/s" if wl.kind == "prefill" else "tokens/s",
+        "ms_per_step": ms_per_step, "steps": steps,
+        "config": workload_config(wl, world, use_graph),
+        "roofline": roofline(dom, work[dom], call_ms[dom], peaks, peaks_src, wl),
+        "step_hbm": step_hbm(work, ms_per_step, peaks),
+        "per_call_ms": call_ms,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+        "wall_s_timed_region": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_baseline(wl, budget_s=cpu_budget)
+    return rec
 
+
+def workload_config(wl, world, use_graph):
+    return {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
+            "H": wl.H, "D": wl.D, "HI": wl.HI, "dI": wl.dI,
+            "l2": "flushed between timed steps (256 MiB write then read, outside the step events)",
+            "launch": "one CUDA graph per step" if use_graph else "direct C-ABI calls",
+            "parallelism": f"dp{world} (independent sequences per GPU)"}
+
+
+def step_hbm(work, ms, peaks):
+    """Algorithmic bytes of the whole step over its time, against the measured
+    copy bandwidth and the 8 TB/s nominal figure."""
+    nbytes = sum(w["bytes"] for w in work.values())
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac_measured": gbs / peaks["hbm_gbs"],
+            "frac_8tbs": gbs / HBM_NOMINAL_GBS}
+
+
+def gpu_arm(args, names):
+    import torch.distributed as dist
+
+    import synth
+
+    world, rank, local, dev = init_ranks()
+    peaks, peaks_src = load_peaks()
+    recs = {}
+    for k, name in enumerate(names):
+        wl = synth.WORKLOADS[name]
+        steps = args.steps if k == 0 else min(args.steps, SECONDARY_STEPS)
+        budget = args.cpu_budget if k == 0 else min(args.cpu_budget, SECONDARY_CPU_BUDGET_S)
+        recs[name] = measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, budget)
     line = None
     if rank == 0:
-        work = op_work(wl)
-        dom = max(call_ms, key=lambda k: call_ms[k])
-        roof = roofline(dom, work[dom], call_ms[dom], peaks, peaks_src, wl)
+        head = recs[names[0]]
         line = {
-            "metric": METRIC, "value": value, "unit": r.unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+            "steps": head["steps"], "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) tokens/logits, E2M1 indexer codes, bf16 queries)",
-            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
-                       "H": wl.H, "D": wl.D, "HI": wl.HI, "dI": wl.dI,
-                       "l2": "flushed between timed steps (256 MiB write then read, outside the step events)",
-                       "launch": "one CUDA graph per step" if use_graph else "direct C-ABI calls",
-                       "parallelism": f"dp{world} (independent sequences per GPU)"},
-            "roofline": roof,
-            "per_call_ms": call_ms,
-            "e2e": e2e,
-            "gpu_launches": launches,
-            "clocks": clk,
-            "wall_s_timed_region": wall,
+            "config": head["config"],
         }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+        for key in ("roofline", "step_hbm", "per_call_ms", "e2e", "gpu_launches", "clocks",
+                    "wall_s_timed_region", "cpu_baseline"):
+            if key in head:
+                line[key] = head[key]
+        if len(names) > 1:
+            line["workloads"] = {n: recs[n] for n in names}
     if world > 1:
         dist.barrier()
-    r.graphs.clear()
-    if world > 1:
         dist.destroy_process_group()
     return line
+
+
+def relaunch_with_ranks(n):
+    """`bench.py --gpus N` started without torchrun: run the same command as N
+    ranks on this node (one per GPU) and return their exit status."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
 
 
 def launch_count():
@@ -486,7 +562,7 @@ def launch_count():
     return csa.launch_count()
 
 
-def e2e_leg(r, args, world, dev, use_graph):
+def e2e_leg(r, args, world, dev, use_graph, steps):
     """The same step through the public API: pinned host inputs copied in and the
     attention output copied back, all inside the timed region."""
     import torch
@@ -509,7 +585,7 @@ def e2e_leg(r, args, world, dev, use_graph):
     step = args.warmup
     g = r.graph(step, inputs=dbuf, key="e2e") if use_graph else None
     times = []
-    for i in range(max(1, min(args.steps, 10)) + 2):
+    for i in range(max(1, min(steps, 10)) + 2):
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
@@ -531,19 +607,28 @@ def e2e_leg(r, args, world, dev, use_graph):
 
 
 def roofline(name, work, ms, peaks, src, wl):
+    """Roofline of the step's dominant call: tensor-bound for the attention of
+    prefill and HCA decode (FLOPs against the measured bf16 peak), HBM-bound
+    otherwise (algorithmic bytes against the measured copy bandwidth, and
+    against the 8 TB/s nominal figure)."""
     sec = ms / 1e3
     traffic = kernel_traffic(name, wl.name)
+    gbs = work["bytes"] / sec / 1e9
     if work["flops"] and wl.kind in ("prefill", "hca_decode") and name.endswith("attend"):
         achieved = work["flops"] / sec / 1e12
         peak = peaks["bf16_tflops"]
         return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "peak_source": f"bf16_tflops ({src})", "traffic": traffic,
-                "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"], "ms": ms}
-    achieved = work["bytes"] / sec / 1e9
+                "algorithmic_flops": work["flops"], "algorithmic_bytes": work["bytes"], "ms": ms,
+                "hbm_gbs": gbs, "hbm_frac_measured": gbs / peaks["hbm_gbs"], "hbm_frac_8tbs": gbs / HBM_NOMINAL_GBS}
     peak = peaks["hbm_gbs"]
-    return {"bound": "hbm", "kernel": name, "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "peak_source": f"hbm_gbs ({src})", "traffic": traffic,
-            "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"], "ms": ms}
+    out = {"bound": "hbm", "kernel": name, "achieved": gbs, "peak": peak, "unit": "GB/s",
+           "frac": gbs / peak, "frac_8tbs": gbs / HBM_NOMINAL_GBS, "peak_source": f"hbm_gbs ({src})",
+           "traffic": traffic, "algorithmic_bytes": work["bytes"], "algorithmic_flops": work["flops"], "ms": ms}
+    if work["flops"]:
+        tf = work["flops"] / sec / 1e12
+        out.update({"tflops": tf, "bf16_frac": tf / peaks["bf16_tflops"]})
+    return out
 
 
 def kernel_traffic(call, workload):
@@ -591,7 +676,13 @@ def source_sha(kernel):
 
 
 class OracleStep:
-    """The oracle's version of one step on a bounded sample of the workload."""
+    """The oracle's version of one step on a bounded sample of the workload.
+
+    Decode samples keep the full context length: the cache before the step
+    holds random finite E4M3 entries (dequantised by the oracle), and only the
+    window tokens and the appended tokens are raw values, so that building the
+    sample stays cheap; the timed step is the oracle's whole step (pool the
+    new tokens, score every visible entry, select, attend)."""
 
     def __init__(self, wl, seed=0, max_seqs=2, max_rows=64):
         import torch
@@ -602,8 +693,7 @@ class OracleStep:
         self.wl = wl
         self.kind = wl.kind
         if wl.kind == "hca_decode":
-            # 1 sequence with a 1/8-length context (1,024 entries): the oracle builds
-            # its cache outside the timed step
+            # 1 sequence with a 1/8-length context (1,024 entries)
             self.B = 1
             T = wl.T // 8
         elif wl.kind in ("decode", "decode_incremental"):
@@ -617,26 +707,26 @@ class OracleStep:
         n_new = wl.m if wl.kind == "hca_decode" else 4
         self.n_new = n_new
         D = wl.D
-        self.x = torch.randn((self.B, T + n_new, D), generator=g).numpy()
-        self.z = torch.randn((self.B, T + n_new, D), generator=g).numpy()
         if wl.kind == "prefill":
+            self.x = torch.randn((self.B, T, D), generator=g).numpy()
+            self.z = torch.randn((self.B, T, D), generator=g).numpy()
             self.rows = np.unique(np.linspace(0, T - 1, min(max_rows, T)).astype(np.int64))
             self.q = synth.queries(self.B, len(self.rows), wl.H, D, wl.q_scale, seed).view(torch.int16).numpy().view(np.uint16)
-            ind = synth.indexer_inputs(self.B, len(self.rows), wl.N, wl.HI, wl.dI, seed)
-        else:
-            self.q = synth.queries(self.B, 1, wl.H, D, wl.q_scale, seed).view(torch.int16).numpy().view(np.uint16)
-            N = (T + n_new) // wl.m
-            ind = synth.indexer_inputs(self.B, 1, N, max(wl.HI, 1), max(wl.dI, 32), seed) if wl.HI else None
-        self.ind = ind
-        if wl.kind != "prefill":
-            # the cache state before the step (built once, untimed)
-            n0 = T // wl.m
-            c, s = ocsa.quantize_entries(ocsa.compress(self.x[:, :T], self.z[:, :T], wl.m))
-            self.entries = np.zeros((self.B, n0 + 1, D))
-            self.entries[:, :n0] = ocsa.dequantize(c, s)
-            self.win = np.zeros((self.B, T + n_new, D))
-            lo = max(0, T - wl.W)
-            self.win[:, lo:T] = ocsa.window_token_values(self.x[:, lo:T])
+            self.ind = synth.indexer_inputs(self.B, len(self.rows), wl.N, wl.HI, wl.dI, seed)
+            return
+        # raw tokens of positions [base, T + n_new): the window before the step and the new tokens
+        self.base = max(0, T - wl.W)
+        self.x = torch.randn((self.B, T + n_new - self.base, D), generator=g).numpy()
+        self.z = torch.randn((self.B, T + n_new - self.base, D), generator=g).numpy()
+        self.q = synth.queries(self.B, 1, wl.H, D, wl.q_scale, seed).view(torch.int16).numpy().view(np.uint16)
+        N = (T + n_new) // wl.m
+        self.ind = synth.indexer_inputs(self.B, 1, N, max(wl.HI, 1), max(wl.dI, 32), seed) if wl.HI else None
+        n0 = T // wl.m
+        codes, scales = synth.e4m3_cache(self.B, n0, D, seed)
+        self.entries = np.zeros((self.B, n0 + 1, D))
+        self.entries[:, :n0] = ocsa.dequantize(codes.numpy(), scales.numpy())
+        self.win = np.zeros((self.B, T + n_new - self.base, D))
+        self.win[:, :T - self.base] = ocsa.window_token_values(self.x[:, :T - self.base])
 
     def units(self):
         return self.B * (len(self.rows) if self.kind == "prefill" else 1)
@@ -652,19 +742,21 @@ class OracleStep:
             pos = self.rows[None].repeat(self.B, 0)
             idx, _ = o.topk(s64, o.n_visible(pos, m, wl.N), wl.K)
             return o.attend(self.q, ent, idx, lambda b, p: win[b, p], pos, wl.W)
-        T, n_new, m = self.T, self.n_new, wl.m
-        new = o.compress(self.x[:, T:T + n_new], self.z[:, T:T + n_new], m)
+        T, n_new, m, base = self.T, self.n_new, wl.m, self.base
+        lo, hi = T - base, T + n_new - base
+        new = o.compress(self.x[:, lo:hi], self.z[:, lo:hi], m)
         c, s = o.quantize_entries(new)
         self.entries[:, T // m] = o.dequantize(c, s)[:, 0]
-        self.win[:, T:T + n_new] = o.window_token_values(self.x[:, T:T + n_new])
+        self.win[:, lo:hi] = o.window_token_values(self.x[:, lo:hi])
         t = T + n_new - 1
         pos = np.full((self.B, 1), t)
         n_ent = (T + n_new) // m
+        win = lambda b, p: self.win[b, p - base]
         if self.kind == "hca_decode":
-            return o.hca_attend(self.q, self.entries, lambda b, p: self.win[b, p], pos, m, wl.W)
+            return o.hca_attend(self.q, self.entries, win, pos, m, wl.W)
         s64 = o.indexer_scores64(self.ind.qI.numpy(), self.ind.w.numpy(), self.ind.kI[:, :n_ent].numpy())
         idx, _ = o.topk(s64, o.n_visible(pos, m, n_ent), wl.K)
-        return o.attend(self.q, self.entries, idx, lambda b, p: self.win[b, p], pos, wl.W)
+        return o.attend(self.q, self.entries, idx, win, pos, wl.W)
 
     def describe(self):
         wl = self.wl
@@ -674,7 +766,8 @@ class OracleStep:
         if self.kind == "hca_decode":
             return (f"1 sequence, context {self.T} tokens (1/8 of the workload's; {self.T // wl.m} entries): "
                     "append 128 tokens + dense attention")
-        return f"{self.B} of {wl.B} sequences, full {self.T}-token context: append 4 tokens + index + top-k + attend"
+        return (f"{self.B} of {wl.B} sequences, full {self.T}-token context (cache of random finite E4M3 "
+                "entries): append 4 tokens + index + top-k + attend")
 
 
 def cpu_cores():
@@ -685,7 +778,7 @@ def cpu_cores():
 
 
 def cpu_baseline(wl, budget_s=15.0):
-    st = OracleStep(wl)
+    st = OracleStep(wl, max_rows=64 if budget_s >= 15.0 else 16)
     st.run()                          # warm (allocations, BLAS threads)
     t0 = time.perf_counter()
     n = 0
@@ -695,24 +788,36 @@ def cpu_baseline(wl, budget_s=15.0):
         if time.perf_counter() - t0 > budget_s or n >= 50:
             break
     dt = (time.perf_counter() - t0) / n
-    return {"value": st.units() / dt, "unit": "tokens/s" if wl.kind != "prefill" else "queries/s",
-            "cores": cpu_cores(), "kind": "oracle", "sample": st.describe(), "sec_per_sample": dt}
+    out = {"value": st.units() / dt, "unit": "tokens/s" if wl.kind != "prefill" else "queries/s",
+           "cores": cpu_cores(), "kind": "oracle", "sample": st.describe(), "sec_per_sample": dt}
+    if wl.kind == "prefill":
+        # the rate of the sampled rows, extrapolated to every row of the workload
+        out["extrapolated"] = True
+        out["extrapolated_full_step_s"] = wl.B * wl.T / out["value"]
+    return out
 
 
-def reference_arm(args, wl):
+def reference_arm(args, wl, others=()):
+    """The oracle timed on the host cores (rank 0 only): `args.steps` steps of
+    the bounded sample of `wl`, plus one step of each workload in `others`."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return None
-    st = OracleStep(wl)
-    for _ in range(args.warmup):
-        st.run()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        st.run()
-    dt = (time.perf_counter() - t0) / args.steps
+
+    def run(w, steps, warmup):
+        st = OracleStep(w)
+        for _ in range(warmup):
+            st.run()
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            st.run()
+        dt = (time.perf_counter() - t0) / steps
+        return st, dt
+
+    st, dt = run(wl, args.steps, args.warmup)
     unit = "tokens/s" if wl.kind != "prefill" else "queries/s"
     value = st.units() / dt
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 0,
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
@@ -720,6 +825,14 @@ def reference_arm(args, wl):
             "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                              "sample": st.describe()},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if others:
+        line["workloads"] = {}
+        for w in others:
+            so, d = run(w, 1, 0)
+            u = "tokens/s" if w.kind != "prefill" else "queries/s"
+            line["workloads"][w.name] = {"value": so.units() / d, "unit": u, "ms_per_step": d * 1e3,
+                                         "sample": so.describe(), "cores": cpu_cores()}
+    return line
 
 
 def kernel_case(args, wl):
@@ -814,9 +927,11 @@ def kernel_case(args, wl):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="csa_decode_64k")
+    ap.add_argument("--workload", default="all",
+                    help="one workload, or 'all' (the 1M-context incremental decode first, then every "
+                         "other configuration)")
     ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -824,20 +939,27 @@ def main():
     ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
                     help="run one library call (index_topk, attend, hca_attend, compress_entry, "
-                         "quantize_mxfp4) alone on "
-                         "inputs of the workload's shape; for profilers")
+                         "quantize_mxfp4, decode_step) alone on inputs of the workload's shape; for profilers")
     args = ap.parse_args()
     import synth
-    wl = synth.WORKLOADS[args.workload]
+    world_env = os.environ.get("WORLD_SIZE")
+    if args.gpus > 1 and world_env is None:
+        sys.exit(relaunch_with_ranks(args.gpus))
+    if world_env is not None and int(world_env) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}")
+    names = ALL_WORKLOADS if args.workload == "all" else (args.workload,)
+    for n in names:
+        if n not in synth.WORKLOADS:
+            sys.exit(f"bench.py: unknown workload {n}")
     if args.kernel_case:
-        kernel_case(args, wl)
+        kernel_case(args, synth.WORKLOADS[names[0]])
         return
     if args.impl == "reference":
-        line = reference_arm(args, wl)
+        line = reference_arm(args, synth.WORKLOADS[names[0]], [synth.WORKLOADS[n] for n in names[1:]])
     else:
         if args.warmup < 3:
             args.warmup = 3
-        line = gpu_arm(args, wl)
+        line = gpu_arm(args, names)
     if line is not None:
         print(json.dumps(line), flush=True)
 

@@ -171,6 +171,19 @@ int check_attend_dims(const char *fn, const csa_dims *d, bool dense) {
 
 }  // namespace
 
+namespace csa {
+int check_index_dims(const char *fn, const csa_dims *d) {
+  if (!d) return fail(CSA_ERR_INVALID, "%s: dims is NULL", fn);
+  if (d->B < 0 || d->Tq < 0 || d->m < 1 || d->n_entries < 0 || d->entry_cap < d->n_entries)
+    return fail(CSA_ERR_INVALID, "%s: bad dims (B=%d Tq=%d m=%d n_entries=%d entry_cap=%lld)", fn, d->B, d->Tq,
+                d->m, d->n_entries, (long long)d->entry_cap);
+  if (d->K < 1 || d->K > 2048) return fail(CSA_ERR_UNSUPPORTED, "%s: K=%d (1..2048)", fn, d->K);
+  if ((d->dI != 32 && d->dI != 64) || d->HI < 1 || d->HI > 8)
+    return fail(CSA_ERR_UNSUPPORTED, "%s: HI=%d dI=%d", fn, d->HI, d->dI);
+  return CSA_OK;
+}
+}  // namespace csa
+
 extern "C" {
 
 int csa_version(void) { return 100; }
@@ -221,12 +234,7 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
                    const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
                    size_t workspace_bytes, csa_stream_t stream) {
   clear_error();
-  if (!d) return fail(CSA_ERR_INVALID, "csa_index_topk: dims is NULL");
-  if (d->B < 0 || d->Tq < 0 || d->m < 1 || d->n_entries < 0 || d->entry_cap < d->n_entries)
-    return fail(CSA_ERR_INVALID, "csa_index_topk: bad dims");
-  if (d->K < 1 || d->K > 2048) return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: K=%d (1..2048)", d->K);
-  if ((d->dI != 32 && d->dI != 64) || d->HI < 1 || d->HI > 8)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk: HI=%d dI=%d", d->HI, d->dI);
+  if (int rc = check_index_dims("csa_index_topk", d)) return rc;
   if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
   if (!qI || !w || !kI || !q_pos || !idx_out) return fail(CSA_ERR_INVALID, "csa_index_topk: NULL buffer");
   if (!aligned16(kI) || ((uintptr_t)qI & 3) || ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) ||

@@ -19,6 +19,8 @@ int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);
 void count_launches(unsigned n);   // bookkeeping for csa_launch_count()
 void clear_error();
+// Host checks of a csa_index_topk shape (CSA_OK or the error, message set).
+int check_index_dims(const char *fn, const csa_dims *d);
 
 // ---------------------------------------------------------------------------
 // device status word (set by kernels, read + cleared by csa_sync_status)

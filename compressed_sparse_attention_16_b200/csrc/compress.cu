@@ -9,7 +9,8 @@
 // efficient inference" (ai-papers.net), section "ハイブリッドアテンションの
 // 仕組み" -- KV entries stored in FP8.
 //
-// The op is HBM-bound: 8 bytes read per (token, channel), 1/m byte written.
+// The op is HBM-bound: 8 bytes read per (token, channel), 1/m byte written
+// (4 bytes read when m = 1: a one-token block needs no gate logits).
 // One group of D/4 threads owns one entry; each thread owns 4 channels and
 // streams the block's tokens with 16-byte loads, keeping a per-channel online
 // softmax (running max, normaliser and weighted sum).  The group then reduces
@@ -69,7 +70,12 @@ compress_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_
   const bool active = (g < groups) && (e < n_total) && !(ring_cap > 0 && i + ring_cap < n_per_seq);
 
   float C[4] = {0.f, 0.f, 0.f, 0.f};
-  if (active) {
+  if (active && m == 1) {
+    // a one-token block: the softmax weight is exactly 1, so C = x and the
+    // gate logits are not read at all
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)D) + lane);
+    C[0] = v.x; C[1] = v.y; C[2] = v.z; C[3] = v.w;
+  } else if (active) {
     const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + lane;
     const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + lane;
     OnlineSoftmax4 sm;

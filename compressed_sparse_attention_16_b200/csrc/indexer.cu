@@ -30,6 +30,17 @@ namespace {
 constexpr uint32_t kMagLo = 0x03020100u;   // 2*|E2M1| for codes 0..3
 constexpr uint32_t kMagHi = 0x0C080604u;   // 2*|E2M1| for codes 4..7
 
+// 16 * w as an integer weight, clamped to [0, 16] so that an off-contract
+// weight (negative, above 1, NaN) can never wrap the unsigned score; `bad` is
+// set when w is not a multiple of 1/16 in [0, 1] (the caller raises
+// STATUS_BAD_WEIGHT for it).
+__device__ __forceinline__ int weight16(float w, bool &bad) {
+  const float f = w * 16.f;
+  const int r = __float2int_rn(f);
+  bad = !((float)r == f && r >= 0 && r <= 16);
+  return min(max(r, 0), 16);
+}
+
 __device__ __forceinline__ int e2m1x2_int(uint32_t code) {   // 2*value of one 4-bit code
   const int mag = (int)((0xC8643210u >> (4 * (code & 7))) & 0xF);
   return (code & 8) ? -mag : mag;
@@ -53,9 +64,9 @@ struct IndexQuery {
                                        bool report) {
 #pragma unroll
     for (int h = 0; h < HI; ++h) {
-      const float w16f = wrow[h] * 16.f;
-      w16[h] = __float2int_rn(w16f);
-      if (report && ((float)w16[h] != w16f || w16[h] < 0 || w16[h] > 16)) raise_status(status, STATUS_BAD_WEIGHT);
+      bool bad;
+      w16[h] = weight16(wrow[h], bad);
+      if (report && bad) raise_status(status, STATUS_BAD_WEIGHT);
 #pragma unroll
       for (int k = 0; k < NW; ++k) {
         const uint32_t word = *reinterpret_cast<const uint32_t *>(qrow + h * (DI / 2) + 4 * k);
@@ -714,10 +725,9 @@ index_scan_tc_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w
   int w16[HI];
 #pragma unroll
   for (int h = 0; h < HI; ++h) {
-    const float f = w[(int64_t)row * HI + h] * 16.f;
-    w16[h] = __float2int_rn(f);
-    if (tid == 0 && split == 0 && ((float)w16[h] != f || w16[h] < 0 || w16[h] > 16))
-      raise_status(status, STATUS_BAD_WEIGHT);
+    bool bad;
+    w16[h] = weight16(w[(int64_t)row * HI + h], bad);
+    if (tid == 0 && split == 0 && bad) raise_status(status, STATUS_BAD_WEIGHT);
   }
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
@@ -1152,10 +1162,9 @@ index_decode_kernel(const __grid_constant__ CUtensorMap kmap, const uint8_t *__r
   int w16[HI];
 #pragma unroll
   for (int h = 0; h < HI; ++h) {
-    const float f = w[(int64_t)row * HI + h] * 16.f;
-    w16[h] = __float2int_rn(f);
-    if (tid == 0 && part == 0 && ((float)w16[h] != f || w16[h] < 0 || w16[h] > 16))
-      raise_status(status, STATUS_BAD_WEIGHT);
+    bool bad;
+    w16[h] = weight16(w[(int64_t)row * HI + h], bad);
+    if (tid == 0 && part == 0 && bad) raise_status(status, STATUS_BAD_WEIGHT);
   }
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
@@ -1530,9 +1539,9 @@ index_prefill_tc_kernel(const uint8_t *__restrict__ qI, const float *__restrict_
     nvis = t < 0 ? 0 : (int)min((t + 1) / m, (int64_t)n_entries);
 #pragma unroll
     for (int h = 0; h < HI; ++h) {
-      const float f = w[(row0 + tid) * HI + h] * 16.f;
-      const int w16 = __float2int_rn(f);
-      if ((float)w16 != f || w16 < 0 || w16 > 16) raise_status(status, STATUS_BAD_WEIGHT);
+      bool bad;
+      const int w16 = weight16(w[(row0 + tid) * HI + h], bad);
+      if (bad) raise_status(status, STATUS_BAD_WEIGHT);
       w64[h] = (float)(4 * w16);
     }
   }

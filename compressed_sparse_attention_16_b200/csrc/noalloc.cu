@@ -14,7 +14,10 @@
 // code cannot use the array's name as a device address, so on the first call
 // on each device the entry point asks the runtime for the array's address
 // (cudaGetSymbolAddress with that device current), checks the result and
-// caches it; later calls reuse the cached address.
+// caches it; later calls reuse the cached address.  The cache is per device
+// ordinal for the life of the process: it does not survive cudaDeviceReset
+// (or anything else that destroys and recreates the device's primary
+// context), after which the cached address would be stale.
 #include <mutex>
 
 #include "common.cuh"
@@ -58,7 +61,9 @@ int csa_index_topk_noalloc(const uint8_t *qI, const float *w, const uint8_t *kI,
                            const int32_t *q_pos, const csa_dims *d, int32_t *idx_out,
                            float *score_out, csa_stream_t stream) {
   csa::clear_error();
-  if (!d) return csa::fail(CSA_ERR_INVALID, "csa_index_topk_noalloc: dims is NULL");
+  // the shape is validated first, exactly as csa_index_topk does, so that the
+  // scratch size below is only ever computed for a valid shape
+  if (int rc = csa::check_index_dims("csa_index_topk_noalloc", d)) return rc;
   const size_t need = csa_index_topk_workspace(d);
   if (need > kScratchBytes)
     return csa::fail(CSA_ERR_UNSUPPORTED,

@@ -126,7 +126,11 @@ int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D
  * s < n_vis = min(floor((t + 1) / m), n_entries).  Its score is
  *     score = sum_h w[b,i,h] * max(0, sum_j qI[b,i,h,j] * kI[b,s,j])
  * computed exactly (E2M1 products are multiples of 1/4; w must be a multiple
- * of 1/16 in [0, 1], so 64*score is an integer below 2^24).  The row's output
+ * of 1/16 in [0, 1], so 64*score is an integer below 2^24).  A weight off
+ * that grid is not an argument error the host can see (w lives on the
+ * device): the kernels round 16*w to the nearest integer, clamp it to
+ * [0, 16] and set a status bit that the next csa_sync_status() reports as
+ * CSA_ERR_INVALID; the row's results are then those of the clamped weights.  The row's output
  * lists the min(K, n_vis) best entries in rank order -- score descending, ties
  * to the lower index -- followed by -1 padding.
  *
@@ -153,17 +157,25 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
  * afterwards, plug-ins that only receive their inputs' and outputs' buffers.
  * Same arguments, results and errors as csa_index_topk, minus the workspace:
  * the scratch is an 8 MiB array inside the library's device image, held by
- * every GPU that loads the library until the process exits.  Shapes whose
- * workspace (csa_index_topk_workspace) exceeds 8 MiB -- e.g. more than 2M
- * (query row x entry) pairs -- are rejected with CSA_ERR_UNSUPPORTED before
- * any launch.  The library allocates nothing and calls no allocating routine.
+ * every GPU that loads the library until the process exits.  The shape is
+ * validated first, exactly as csa_index_topk does; a valid shape whose
+ * csa_index_topk_workspace(d) exceeds 8 MiB is then rejected with
+ * CSA_ERR_UNSUPPORTED before any launch.  What fits depends on the path the
+ * shape takes: up to 64 query rows with >= 2,048 entries, 4 bytes per
+ * (row, entry) plus 32 KiB per row (16 rows x 16,384 entries: 1.5 MiB;
+ * 64 rows x 20,000 entries: 7.2 MiB); 65 to 148 decode rows, about 33 KiB
+ * per row; the prefill path (> 64 rows, <= 65,535 entries), 4 bytes per
+ * (row, K), i.e. up to 4,096 rows at K = 512.  The library allocates nothing
+ * and calls no allocating routine.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *     stream capture.  The cached address does not survive cudaDeviceReset
+ *     (or any destruction of the device's primary context).
  *   - All calls share the one array: calls whose kernels overlap on the GPU
  *     (different streams, or different host threads) race and corrupt each
  *     other's results; serialise them.  Stale contents from an earlier call
- *     are harmless (every score is written before it is read).
+ *     are harmless (every score is written before it is read, and the
+ *     counters a path needs are cleared by the call itself).
  */
 int csa_index_topk_noalloc(const uint8_t *qI, const float *w, const uint8_t *kI,
                            const int32_t *q_pos, const csa_dims *d, int32_t *idx_out,
