@@ -73,6 +73,10 @@ def op_work(wl):
             items = K + W
             w["attend"] = dict(bytes=B * items * ent + 2 * B * H * D * 2 + B * K * 4 + B * H * 4,
                                flops=4.0 * B * H * items * D)
+            # the fused step moves exactly what the four calls move (the
+            # selection is handed over on chip instead of through memory)
+            w["decode_step"] = dict(bytes=sum(v["bytes"] for v in w.values()),
+                                    flops=sum(v["flops"] for v in w.values()), aggregate=True)
     else:   # prefill
         T, N = wl.T, wl.N
         w["compress_entry"] = dict(bytes=B * T * D * 8 + B * N * ent, flops=0)
@@ -160,7 +164,7 @@ class Runner:
     """One workload's device state.  `calls(i)` lists the library calls of step i
     as (name, launch) pairs; a step is replayed as one CUDA graph."""
 
-    def __init__(self, wl, seed, device):
+    def __init__(self, wl, seed, device, fused=True):
         import torch
 
         import synth
@@ -186,6 +190,11 @@ class Runner:
             if not dense:
                 self.ind = synth.indexer_inputs(wl.B, 1, cap, wl.HI, wl.dI, seed, device=device)
                 self.state.kI.copy_(self.ind.kI)
+                # each step's new tokens as contiguous [B, n_new, D] blocks (the fused step's input)
+                steps_x = self.x[:, self.T0:self.T0 + self.n_new * self.n_steps]
+                steps_z = self.z[:, self.T0:self.T0 + self.n_new * self.n_steps]
+                self.x_steps = steps_x.reshape(wl.B, self.n_steps, self.n_new, wl.D).transpose(0, 1).contiguous()
+                self.z_steps = steps_z.reshape(wl.B, self.n_steps, self.n_new, wl.D).transpose(0, 1).contiguous()
             self.q = synth.queries(wl.B, 1, wl.H, wl.D, wl.q_scale, seed, device=device)
             self.state.prefill_context(self.x, self.z, self.T0)
             # per-step query positions (graph-static)
@@ -196,6 +205,7 @@ class Runner:
             self.Dims = Dims
             # workspaces sized for the largest step, allocated before any capture
             import compressed_sparse_attention_16_b200 as csa
+            self.fused = False
             for j in (0, self.n_steps - 1):
                 d = self._dims(j)
                 if wl.kind == "hca_decode":
@@ -203,6 +213,12 @@ class Runner:
                 else:
                     self._ws(csa.index_topk_workspace(d), "_ws_index")
                     self._ws(csa.attend_workspace(d), "_ws_attend")
+                    nb = csa.decode_step_workspace(d, self.n_new) if fused else 0
+                    if nb:
+                        self.fused = True
+                        if getattr(self, "_ws_step", None) is None or self._ws_step.numel() < nb:
+                            # zero-filled once: the fused step keeps its barrier words consistent
+                            self._ws_step = torch.zeros(nb + 4096, dtype=torch.uint8, device=device)
         else:
             self.x, self.z = synth.tokens(wl.B, wl.T, wl.D, seed, device=device)
             self.q = synth.queries(wl.B, wl.T, wl.H, wl.D, wl.q_scale, seed, device=device)
@@ -287,6 +303,15 @@ class Runner:
             ws = self._ws(csa.attend_workspace(d, True), "_ws_hca")
             out.append(("hca_attend", lambda: csa.hca_attend(q, st.codes, st.scales, st.win_codes, st.win_scales,
                                                              q_pos, d, st.out, st.lse, workspace=ws)))
+        elif self.fused:
+            qI = self.ind.qI if inputs is None else inputs["qI"]
+            w = self.ind.w if inputs is None else inputs["w"]
+            xs = self.x_steps[j] if inputs is None else inputs["x"]
+            zs = self.z_steps[j] if inputs is None else inputs["z"]
+            ws = self._ws_step
+            return [("decode_step", lambda: csa.decode_step(xs, zs, None, q, qI, w, q_pos, st.codes, st.scales, st.kI,
+                                                            st.win_codes, st.win_scales, d, st.idx, st.score, st.out,
+                                                            st.lse, ws))]
         else:
             qI = self.ind.qI if inputs is None else inputs["qI"]
             w = self.ind.w if inputs is None else inputs["w"]
@@ -309,6 +334,9 @@ class Runner:
         only the attention, so they run on a side stream beside the indexer
         (CSA) or beside each other (HCA); the attention waits for both."""
         torch = self.torch
+        if len(calls) == 1:               # the fused decode step: one launch
+            calls[0][1]()
+            return
         if self._side is None:
             self._side = torch.cuda.Stream(device=self.dev)
         side, main = self._side, torch.cuda.current_stream(self.dev)
@@ -404,7 +432,7 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     import torch
     import torch.distributed as dist
 
-    r = Runner(wl, seed=rank, device=dev)
+    r = Runner(wl, seed=rank, device=dev, fused=not args.unfused)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     use_graph = r.decode and not args.no_graph
 
@@ -469,6 +497,7 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     call_ms = {k: float(np.mean([a.elapsed_time(b) for a, b in v])) for k, v in per_call.items()}
 
     e2e = e2e_leg(r, args, world, dev, use_graph, steps)
+    fused = getattr(r, "fused", False)
     r.graphs.clear()
     del r, flush
     torch.cuda.empty_cache()
@@ -479,7 +508,7 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     rec = {
         "value": value, "unit": "queries/s" if wl.kind == "prefill" else "tokens/s",
         "ms_per_step": ms_per_step, "steps": steps,
-        "config": workload_config(wl, world, use_graph),
+        "config": workload_config(wl, world, use_graph, fused),
         "roofline": roofline(dom, work[dom], call_ms[dom], peaks, peaks_src, wl),
         "step_hbm": step_hbm(work, ms_per_step, peaks),
         "per_call_ms": call_ms,
@@ -493,18 +522,19 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     return rec
 
 
-def workload_config(wl, world, use_graph):
+def workload_config(wl, world, use_graph, fused=False):
     return {"workload": wl.name, "B": wl.B, "T": wl.T, "m": wl.m, "K": wl.K, "W": wl.W,
             "H": wl.H, "D": wl.D, "HI": wl.HI, "dI": wl.dI,
             "l2": "flushed between timed steps (256 MiB write then read, outside the step events)",
-            "launch": "one CUDA graph per step" if use_graph else "direct C-ABI calls",
+            "launch": ("one CUDA graph per step" if use_graph else "direct C-ABI calls")
+            + (" of one csa_decode_step launch" if fused else ""),
             "parallelism": f"dp{world} (independent sequences per GPU)"}
 
 
 def step_hbm(work, ms, peaks):
     """Algorithmic bytes of the whole step over its time, against the measured
     copy bandwidth and the 8 TB/s nominal figure."""
-    nbytes = sum(w["bytes"] for w in work.values())
+    nbytes = sum(w["bytes"] for w in work.values() if not w.get("aggregate"))
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"algorithmic_bytes": nbytes, "achieved_gbs": gbs, "frac_measured": gbs / peaks["hbm_gbs"],
             "frac_8tbs": gbs / HBM_NOMINAL_GBS}
@@ -936,6 +966,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run CSA decode steps as the separate calls instead of one csa_decode_step launch")
     ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
                     help="run one library call (index_topk, attend, hca_attend, compress_entry, "

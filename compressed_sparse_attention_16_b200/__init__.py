@@ -40,6 +40,8 @@ SYMBOLS = (
     "csa_launch_count",
     "csa_quantize_mxfp4",
     "csa_selftest_timeout",
+    "csa_decode_step_workspace",
+    "csa_decode_step",
 )
 
 
@@ -110,6 +112,11 @@ def lib() -> ctypes.CDLL:
     L.csa_selftest_timeout.restype = ctypes.c_int
     L.csa_quantize_mxfp4.argtypes = [_P, _I64, _I32, _P, _P, _P]
     L.csa_quantize_mxfp4.restype = ctypes.c_int
+    L.csa_decode_step_workspace.argtypes = [ctypes.POINTER(Dims), _I32]
+    L.csa_decode_step_workspace.restype = _SZ
+    L.csa_decode_step.argtypes = [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(Dims),
+                                  _P, _P, _P, _P, _P, _SZ, _P]
+    L.csa_decode_step.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -250,6 +257,34 @@ def hca_attend(q, codes, scales, win_codes, win_scales, q_pos, dims: Dims, out, 
                             _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
                             _ptr(out, torch.bfloat16, "out", dev), _ptr(lse, torch.float32, "lse", dev),
                             wp, wn, _stream(stream)))
+
+
+def decode_step_workspace(dims: Dims, n_new: int) -> int:
+    """Bytes of workspace csa_decode_step needs (0: the shape is outside the
+    fused step's set; use the separate calls)."""
+    return int(lib().csa_decode_step_workspace(ctypes.byref(dims), int(n_new)))
+
+
+def decode_step(x_new, z_new, kI_new, q, qI, w, q_pos, codes, scales, kI, win_codes, win_scales,
+                dims: Dims, idx_out, score_out, out, lse, workspace, stream=None) -> None:
+    """csa_decode_step: append x_new/z_new [B, n, D] (and kI_new [B, n/m, dI/2]
+    or None), then index, select and attend for one query per sequence, in one
+    launch; see include/csa.h.  `workspace` (u8, >= decode_step_workspace
+    bytes) must have been zero-filled before its first use."""
+    dev = q.device
+    if x_new.dim() != 3 or z_new.shape != x_new.shape:
+        raise ValueError("x_new and z_new must be [B, n_new, D] of equal shape")
+    _check(lib().csa_decode_step(
+        _ptr(x_new, torch.float32, "x_new", dev), _ptr(z_new, torch.float32, "z_new", dev), x_new.shape[1],
+        _ptr(kI_new, torch.uint8, "kI_new", dev), _ptr(q, torch.bfloat16, "q", dev),
+        _ptr(qI, torch.uint8, "qI", dev), _ptr(w, torch.float32, "w", dev), _ptr(q_pos, torch.int32, "q_pos", dev),
+        _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
+        _ptr(kI, torch.uint8, "kI", dev), _ptr(win_codes, torch.uint8, "win_codes", dev),
+        _ptr(win_scales, torch.float32, "win_scales", dev), ctypes.byref(dims),
+        _ptr(idx_out, torch.int32, "idx_out", dev), _ptr(score_out, torch.float32, "score_out", dev),
+        _ptr(out, torch.bfloat16, "out", dev), _ptr(lse, torch.float32, "lse", dev),
+        _ptr(workspace, torch.uint8, "workspace", dev), workspace.numel() if workspace is not None else 0,
+        _stream(stream)))
 
 
 def sync_status(stream=None) -> None:

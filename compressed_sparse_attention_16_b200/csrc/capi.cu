@@ -23,6 +23,12 @@ int launch_attend(const uint16_t *q, const uint8_t *codes, const float *scales, 
                   const csa_dims *d, uint16_t *out, float *lse, void *workspace, size_t ws_bytes,
                   cudaStream_t stream);
 size_t attend_workspace(const csa_dims *d, bool dense);
+size_t decode_step_workspace(const csa_dims *d, int n_new);
+int launch_decode_step(const float *x_new, const float *z_new, int n_new, const uint8_t *kI_new,
+                       const uint16_t *q, const uint8_t *qI, const float *w, const int32_t *q_pos,
+                       uint8_t *codes, float *scales, uint8_t *kI, uint8_t *win_codes, float *win_scales,
+                       const csa_dims *d, int32_t *idx_out, float *score_out, uint16_t *out, float *lse,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
 // errors
@@ -293,6 +299,36 @@ int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
                size_t workspace_bytes, csa_stream_t stream) {
   return attend_common("hca_attend", q, codes, scales, nullptr, win_codes, win_scales, q_pos, d,
                        out, lse, workspace, workspace_bytes, stream);
+}
+
+size_t csa_decode_step_workspace(const csa_dims *d, int32_t n_new) {
+  if (!d) return 0;
+  const size_t n = decode_step_workspace(d, n_new);
+  clear_error();
+  return n;
+}
+
+int csa_decode_step(const float *x_new, const float *z_new, int32_t n_new, const uint8_t *kI_new,
+                    const uint16_t *q, const uint8_t *qI, const float *w, const int32_t *q_pos,
+                    uint8_t *codes, float *scales, uint8_t *kI, uint8_t *win_codes, float *win_scales,
+                    const csa_dims *d, int32_t *idx_out, float *score_out, uint16_t *out, float *lse,
+                    void *workspace, size_t workspace_bytes, csa_stream_t stream) {
+  clear_error();
+  if (int rc = check_index_dims("csa_decode_step", d)) return rc;
+  if (int rc = check_attend_dims("csa_decode_step", d, false)) return rc;
+  if (d->B == 0) return CSA_OK;
+  if (!x_new || !z_new || !q || !qI || !w || !q_pos || !codes || !scales || !kI || !win_codes || !win_scales ||
+      !idx_out || !out)
+    return fail(CSA_ERR_INVALID, "csa_decode_step: NULL buffer");
+  if (!aligned16(x_new) || !aligned16(z_new) || !aligned16(q) || !aligned16(out) || !aligned16(codes) ||
+      !aligned16(kI) || !aligned16(win_codes) || (kI_new && !aligned16(kI_new)) || ((uintptr_t)qI & 15) ||
+      ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) || ((uintptr_t)scales & 3) || ((uintptr_t)win_scales & 3) ||
+      ((uintptr_t)idx_out & 3) || ((uintptr_t)score_out & 3) || ((uintptr_t)lse & 3) || !aligned16(workspace))
+    return fail(CSA_ERR_INVALID, "csa_decode_step: misaligned buffer");
+  if (int rc = need_status()) return rc;
+  return launch_decode_step(x_new, z_new, n_new, kI_new, q, qI, w, q_pos, codes, scales, kI, win_codes, win_scales,
+                            d, idx_out, score_out, out, lse, workspace, workspace_bytes,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 int csa_sync_status(csa_stream_t stream) {

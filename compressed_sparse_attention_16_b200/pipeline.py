@@ -10,7 +10,8 @@ current CUDA stream.
 * :class:`DecodeState` -- a decode-time cache (compressed entries, indexer
   keys, a window ring of ``win_cap`` tokens) that grows by one compressed
   entry per ``m`` appended tokens, with :meth:`DecodeState.step` running one
-  append + query step (CSA: index, top-k, attend; HCA: dense attend).
+  append + query step (CSA: index, top-k, attend -- one fused launch when the
+  shape allows it; HCA: dense attend).
 """
 from __future__ import annotations
 
@@ -18,7 +19,8 @@ import dataclasses
 
 import torch
 
-from . import Dims, attend, attend_workspace, compress, hca_attend, index_topk, index_topk_workspace
+from . import (Dims, attend, attend_workspace, compress, decode_step, decode_step_workspace, hca_attend, index_topk,
+               index_topk_workspace)
 
 
 def _ws(nbytes: int, device) -> torch.Tensor | None:
@@ -73,11 +75,14 @@ class DecodeState:
     window ring.  Capacity is fixed at construction (``entry_cap`` entries).
 
     ``dense=True`` makes it an HCA cache (no indexer, dense attention).
+    ``fused=True`` (the default) runs each CSA step as one csa_decode_step
+    launch where the shape allows it; ``fused=False`` always uses the
+    separate calls.
     """
 
     def __init__(self, B: int, D: int, H: int, m: int, W: int, entry_cap: int, *, K: int = 512,
                  HI: int = 4, dI: int = 64, win_cap: int | None = None, dense: bool = False,
-                 softmax_scale: float = 1.0, device="cuda"):
+                 softmax_scale: float = 1.0, device="cuda", fused: bool = True):
         self.B, self.D, self.H, self.m, self.W, self.K = B, D, H, m, W, K
         self.HI, self.dI, self.dense = HI, dI, dense
         self.win_cap = W if win_cap is None else win_cap
@@ -98,16 +103,29 @@ class DecodeState:
         self.lse = torch.empty((B, 1, H), dtype=torch.float32, device=dev)
         self._ws_index = None
         self._ws_attend = None
+        self._ws_step = None
         self._side = None
+        self.fused = fused and not dense
 
     @property
     def n_entries(self) -> int:
         return self.n_tokens // self.m
 
-    def dims(self) -> Dims:
+    def dims(self, n_tokens: int | None = None) -> Dims:
+        n = self.n_tokens if n_tokens is None else n_tokens
         return Dims(B=self.B, Tq=1, H=self.H, D=self.D, HI=self.HI, dI=self.dI, K=self.K, W=self.W,
-                    m=self.m, n_entries=self.n_entries, entry_cap=self.entry_cap,
+                    m=self.m, n_entries=n // self.m, entry_cap=self.entry_cap,
                     win_cap=self.win_cap, softmax_scale=self.softmax_scale)
+
+    def step_workspace(self, n_new: int) -> torch.Tensor | None:
+        """The zero-filled workspace of the fused step for n_new appended
+        tokens (grown when needed), or None if the shape is not fused."""
+        nb = decode_step_workspace(self.dims(self.n_tokens + n_new), n_new)
+        if not nb:
+            return None
+        if self._ws_step is None or self._ws_step.numel() < nb:
+            self._ws_step = torch.zeros(nb, dtype=torch.uint8, device=self.device)
+        return self._ws_step
 
     def prefill_context(self, x: torch.Tensor, z: torch.Tensor, T: int, kI: torch.Tensor | None = None):
         """Compress tokens [0, T) of x, z [B, >=T, D] into the cache (setup).
@@ -170,12 +188,25 @@ class DecodeState:
     def step(self, x_new, z_new, q, qI=None, w=None, kI_new=None):
         """Append tokens then run one query per sequence at the newest position.
 
-        CSA: the new entries' indexer keys are stored first; the compression
+        CSA: one csa_decode_step launch (append, index, select, attend) when
+        the shape is in its set and ``fused`` is on.  Otherwise the separate
+        calls: the new entries' indexer keys are stored first; the compression
         of the new tokens (needed only by the attention) runs on a side stream
         beside the indexer, and the attention waits for both."""
         if self.dense:
             self.append(x_new, z_new, kI_new)
             return self.query(q, qI, w)
+        n = x_new.shape[1]
+        ws = self.step_workspace(n) if self.fused else None
+        if ws is not None:
+            assert self.n_tokens % self.m == 0 and n % self.m == 0
+            assert (self.n_tokens + n) // self.m <= self.entry_cap
+            self.q_pos.fill_(self.n_tokens + n - 1)
+            decode_step(x_new, z_new, kI_new, q, qI, w, self.q_pos, self.codes, self.scales, self.kI,
+                        self.win_codes, self.win_scales, self.dims(self.n_tokens + n), self.idx, self.score,
+                        self.out, self.lse, ws)
+            self.n_tokens += n
+            return self.out, self.lse
         main = torch.cuda.current_stream(self.device)
         if self._side is None:
             self._side = torch.cuda.Stream(device=self.device)

@@ -221,6 +221,63 @@ int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
                const csa_dims *d, uint16_t *out, float *lse, void *workspace,
                size_t workspace_bytes, csa_stream_t stream);
 
+/*
+ * csa_decode_step -- one whole CSA decode step in a single launch: append the
+ * step's new tokens, then index, select and attend for one query per
+ * sequence.
+ * (jiwasawa.github.io DeepSeek-V4 article, "Compressed Sparse Attention
+ *  (CSA)": indexer scores, top-k selector, shared key-value MQA over the
+ *  selected entries; "Heavily Compressed Attention (HCA)": the sliding-window
+ *  branch; hazakura.dev "衝撃1：CSA + HCA": 4 tokens per entry, FP4 indexer,
+ *  128-token window, 1M-token contexts; studioglobal.ai "アテンションの
+ *  ブレイクスルー": softmax-gated pooling, top 512 blocks.)
+ *
+ * Computes exactly what this sequence of calls computes, for every sequence
+ * b with query position t = q_pos[b]:
+ *   1. csa_compress of the n_new tokens x_new/z_new[b] (positions
+ *      t - n_new + 1 .. t, which must end a block: (t + 1) % m == 0) into the
+ *      entries (t + 1)/m - n_new/m .. (t + 1)/m - 1 of codes/scales, and with
+ *      m = 1 into the window ring win_codes/win_scales (slot p % win_cap);
+ *   2. if kI_new is not NULL, its rows are copied into kI at those entries;
+ *   3. csa_index_topk (Tq = 1) -> idx_out, score_out;
+ *   4. csa_attend -> out, lse.
+ * The results are bit-identical to those calls' (the same arithmetic in the
+ * same order).  A query position that does not end a block, or that has
+ * fewer than n_new tokens before it, skips the append for that sequence and
+ * sets a status bit (csa_sync_status -> CSA_ERR_INVALID).
+ *
+ *   x_new, z_new  fp32 [B, n_new, D]
+ *   kI_new        u8 [B, n_new / m, dI / 2] packed E2M1, or NULL (keys already in kI)
+ *   q             bf16 [B, 1, H, D];  qI u8 [B, 1, HI, dI/2] (16-byte aligned);  w fp32 [B, 1, HI]
+ *   q_pos         int32 [B]
+ *   codes, scales, kI, win_codes, win_scales: the caches of csa_compress /
+ *                 csa_index_topk / csa_attend, updated in place
+ *   d             the csa_index_topk / csa_attend shape: Tq = 1, n_entries =
+ *                 the entry count after the append (visibility is capped by it)
+ *   idx_out int32 [B, 1, K];  score_out fp32 [B, 1, K] or NULL
+ *   out bf16 [B, 1, H, D];  lse fp32 [B, 1, H] or NULL
+ *   workspace     at least csa_decode_step_workspace(d, n_new) bytes.  It must
+ *                 be zero-filled once before its first use (cudaMemset after
+ *                 allocation); every call leaves the words that carry its grid
+ *                 barriers in the state the next call expects, and zeroes its
+ *                 own counters.  After a call that timed out (csa_sync_status
+ *                 returns CSA_ERR_TIMEOUT) zero it again.  Calls that share a
+ *                 workspace must not overlap on the GPU.
+ * Supported: H = 128, D = 512, dI = 64, HI <= 4, Tq = 1, K <= 2048, n_new a
+ * multiple of m with n_new <= 16 and n_new <= win_cap, 2*B <= the GPU's SM
+ * count, at most 8,192 visible entries per CTA (B sequences share the SMs).
+ * Anything else returns CSA_ERR_UNSUPPORTED before any launch (use the
+ * separate calls); csa_decode_step_workspace returns 0 for such shapes.
+ * The launch is cooperative (one CTA per SM); it must not be issued while
+ * another kernel occupies the GPU's SMs indefinitely.
+ */
+size_t csa_decode_step_workspace(const csa_dims *d, int32_t n_new);
+int csa_decode_step(const float *x_new, const float *z_new, int32_t n_new, const uint8_t *kI_new,
+                    const uint16_t *q, const uint8_t *qI, const float *w, const int32_t *q_pos,
+                    uint8_t *codes, float *scales, uint8_t *kI, uint8_t *win_codes, float *win_scales,
+                    const csa_dims *d, int32_t *idx_out, float *score_out, uint16_t *out, float *lse,
+                    void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 const char *csa_last_error(void);
 
