@@ -432,7 +432,7 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     import torch
     import torch.distributed as dist
 
-    r = Runner(wl, seed=rank, device=dev, fused=not args.unfused)
+    r = Runner(wl, seed=rank, device=dev, fused=args.decode_path == "fused")
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     use_graph = r.decode and not args.no_graph
 
@@ -966,8 +966,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
-    ap.add_argument("--unfused", action="store_true",
-                    help="run CSA decode steps as the separate calls instead of one csa_decode_step launch")
+    ap.add_argument("--decode-path", default="fused", choices=["separate", "fused"],
+                    help="CSA decode steps as the separate calls (compress, index_topk, attend) or as one "
+                         "csa_decode_step launch")
     ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
                     help="run one library call (index_topk, attend, hca_attend, compress_entry, "

@@ -288,8 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     for (int c = 0; c < nloc && ok; ++c) {
       const int buf = c & 1;
       // kv_full orders the loaders' scale writes before this thread's reads
-      if (!wait_bar(&bars[BAR_KV_FULL + buf], (c >> 1) & 1, misc, a.status) ||
-          !wait_bar(&bars[BAR_S_FULL + buf], (c >> 1) & 1, misc, a.status)) { ok = false; break; }
+      // one decision per warp: the TMEM accesses and votes below are warp-collective
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[BAR_KV_FULL + buf], (c >> 1) & 1, misc, a.status) &&
+                                       wait_bar(&bars[BAR_S_FULL + buf], (c >> 1) & 1, misc, a.status))) {
+        ok = false;
+        break;
+      }
       tc::fence_after_sync();
       uint32_t sr[32];
       tc::tmem_ld32(tbase + lane_off + TCOL_S + buf * CH, sr);
@@ -305,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       const bool need = mx > m_used + kRescaleLog2;
       if (c > 0 && __any_sync(0xffffffffu, need)) {
         // O holds earlier chunks: wait for the last PV, then rescale this warp's rows
-        if (!wait_bar(&bars[BAR_PV_DONE], (c - 1) & 1, misc, a.status)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, wait_bar(&bars[BAR_PV_DONE], (c - 1) & 1, misc, a.status))) { ok = false; break; }
         tc::fence_after_sync();
         const float f = need ? exp2f(m_used - mx) : 1.f;
 #pragma unroll 1
@@ -343,7 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     }
     // epilogue
     const int64_t orow = (int64_t)row * TH + h;
-    const bool have = nloc > 0 && ok && wait_bar(&bars[BAR_PV_DONE], (nloc - 1) & 1, misc, a.status);
+    // FIN completes once, after every MMA of the CTA (a parity wait on
+    // PV_DONE could see a phase from chunks earlier when the PV MMAs lag)
+    const bool have = __all_sync(0xffffffffu, nloc > 0 && ok && wait_bar(&bars[BAR_FIN], 0, misc, a.status));
     tc::fence_after_sync();
     if (a.splits == 1) {
       if (have) {

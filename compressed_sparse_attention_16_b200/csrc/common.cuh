@@ -40,6 +40,10 @@ int set_smem_once(const void *kernel, int bytes, const char *name);
 // missing or the encoder rejects the arguments.
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner, uint64_t rows,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+// 3-D tensor map without swizzling: dims[0] is the contiguous dimension,
+// strides[0..1] the byte strides of dims 1 and 2, box[0..2] the box.
+bool encode_tmap_3d(CUtensorMap *map, CUtensorMapDataType type, const void *base, const uint64_t dims[3],
+                    const uint64_t strides[2], const uint32_t box[3]);
 
 __device__ __forceinline__ void raise_status(unsigned *status, unsigned bit) {
   atomicOr(status, bit);

@@ -29,21 +29,26 @@
 //       free, and the unit's window rows are prefetched into L2.
 //   A2  select: row histograms in the workspace give the threshold bin; the
 //       keys at or above it become candidates (unique 64-bit keys score,
-//       ~index), with an exact refinement when ties flood the bin; every
-//       candidate is ranked by counting the larger ones, and the K best are
-//       written in rank order.
-//   B   attend: every CTA becomes one attention unit (sequence, half of D,
-//       item split) and runs the tensor-core MQA over its chunks of the
-//       sequence's item list (selected entries, then window tokens): E4M3 rows
-//       converted exactly to bf16, S = Q K^T (M = 128 heads, N = 32 items,
-//       K = 512) and O += P V (N = 256) in TMEM, online softmax with lazy
-//       rescaling; item splits write unnormalised partials that one more grid
-//       barrier lets every unit merge for its share of the heads.
+//       ~index, their cache rows prefetched into L2), with an exact
+//       refinement when ties flood the bin; every candidate is ranked by
+//       counting the larger ones (the row's CTAs share the candidates), and
+//       the K best are written in rank order.
+//   B   attend: every CTA becomes one attention unit (sequence, quarter of
+//       D, item split) and runs the tensor-core MQA over its chunks of the
+//       sequence's item list (selected entries, then window tokens).  Q lives
+//       in TMEM as the A operand of S = Q K^T (M = 128 heads, N = 32 items,
+//       K = 512), so the tensor core streams only the item tile from shared
+//       memory; E4M3 rows are converted exactly to bf16; the softmax (one head
+//       per thread, lazy rescaling) writes P = p * item scale straight into
+//       TMEM as the A operand of O += P V (N = 128, the unit's quarter of D).
+//       Item splits write unnormalised partials and count themselves done
+//       per (sequence, quarter); each unit then merges its share of the heads.
 //
 // Grid barriers count arrivals on a 64-bit word that only ever grows by one
-// per CTA and barrier, so a workspace needs zero filling once, before its
-// first use; the per-call counters are zeroed by the kernel itself (before a
-// barrier that precedes their first use).
+// per CTA and barrier, and the per-(sequence, quarter) merge counters only
+// grow too; the per-call selection counters are cleared by each call after
+// their last use.  So a workspace needs zero filling once, before its first
+// use, and again only when the shape changes or a call timed out.
 // Every wait is bounded by wall time; on expiry the kernel sets the status
 // word's timeout bit, stops waiting, and unwinds.
 #include "common.cuh"
@@ -66,10 +71,11 @@ constexpr unsigned long long kWaitNs = 2000000000ull;
 
 constexpr int TH = 128;                // attention heads = MMA M
 constexpr int TD = 512;                // entry width
-constexpr int CH = 32;                 // items per chunk = QK MMA N
-constexpr int DHALF = 256;             // output columns per unit = PV MMA N
+constexpr int CH = 128;                // items per chunk = QK MMA N
+constexpr int DQ = 128;                // output columns per unit (a quarter of D) = PV MMA N
 constexpr int kMaxSelLocal = 2304;     // selected items one unit may hold
 constexpr int kMaxNew = 16;            // appended tokens per step
+constexpr int kMaxSplits = 64;         // item splits per (sequence, quarter) at most
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
 
@@ -79,28 +85,36 @@ constexpr uint32_t A_SC = A_KBUF + kStages * kBatchBytes;       // u32 scores; l
 constexpr uint32_t A_HIST = A_SC + kLocalCap * 4;               // u32 [4096]
 constexpr uint32_t A_QI = A_HIST + kBins * 4;                   // indexer queries (MMA B operand)
 constexpr uint32_t A_END = A_QI + 256;
-constexpr uint32_t B_Q = 0;                                     // 128 x 512 bf16, 32 TMA boxes
-constexpr uint32_t B_KV = B_Q + TH * TD * 2;                    // 2 x 32 items x 512 bf16
-constexpr uint32_t KV_BYTES = CH * TD * 2;
-constexpr uint32_t B_P = B_KV + 2 * KV_BYTES;                   // 2 x 128 heads x 32 bf16
-constexpr uint32_t P_BYTES = TH * CH * 2;
-constexpr uint32_t B_SEL = B_P + 2 * P_BYTES;                   // int32 [kMaxSelLocal]
-constexpr uint32_t B_SCALE = B_SEL + kMaxSelLocal * 4;          // fp32 [2][32]
-constexpr uint32_t B_END = B_SCALE + 2 * CH * 4;
+// Q is staged at 0 (TMA: [32 d-blocks][128 heads][16 d] bf16) and moved into
+// TMEM; the region then holds the item tile [128 items][512 d] bf16.
+constexpr uint32_t B_Q = 0;
+constexpr uint32_t B_KV = 0;
+constexpr uint32_t KV_BYTES = CH * TD * 2;                      // 128 KiB
+constexpr uint32_t B_P = B_KV + KV_BYTES;                       // P [128 heads][128 items] bf16
+constexpr uint32_t P_BYTES = TH * CH * 2;                       // 32 KiB
+constexpr uint32_t B_SEL = B_P + P_BYTES;                       // int32 [kMaxSelLocal]
+constexpr uint32_t B_SCALE = B_SEL + kMaxSelLocal * 4;          // fp32 [128] item scales
+constexpr uint32_t B_MX = B_SCALE + CH * 4;                     // fp32 [2][128] per-half maxima / sums
+constexpr uint32_t B_END = B_MX + 2 * TH * 4;
 constexpr uint32_t OFF_BAR = ((A_END > B_END ? A_END : B_END) + 127u) & ~127u;
-constexpr int NBAR = 17;
+constexpr int NBAR = 15;
 constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127u) & ~127u;
 
-enum { A_FULL = 0, A_MDONE = 4, BAR_KV_FULL = 6, BAR_KV_FREE = 8, BAR_S_FULL = 10, BAR_P_FULL = 12,
-       BAR_PV_DONE = 14, BAR_FIN = 15, BAR_Q = 16 };
+enum { A_FULL = 0, A_MDONE = 4, BAR_KV_FULL = 6, BAR_KV_FREE = 7, BAR_S_FULL = 8, BAR_P_FULL = 9,
+       BAR_PV_DONE = 10, BAR_FIN = 11, BAR_Q = 12, BAR_QT = 13, BAR_MX = 14 };
 
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TCOL_SFA = 128, TCOL_SFB = 132;   // scan: accumulators at 0..127
-constexpr uint32_t TCOL_O = 0, TCOL_S = 256;         // attention
+// attention: Q (bf16, the A operand of S = Q K^T), S of the current chunk,
+// the unit's quarter of O
+constexpr uint32_t TCOL_Q = 0, TCOL_S = 256, TCOL_O = 384;
 
 struct Misc {
   unsigned long long base_ctr;  // grid-barrier counter at the start of this call
   uint32_t nbar;                // grid barriers this CTA has arrived at
+  uint32_t pair_base;           // this unit's pair counter at the start of this call
+  uint32_t cbase_a, cbase_b;    // candidate counters of the scan row and the unit's row at the start
+  uint32_t token;               // this call's token (never 0)
   uint32_t tmem;
   int abort;
   int bin;
@@ -119,13 +133,14 @@ struct Ws {
   uint32_t zone_u4;   // their size in 16-byte words
   uint32_t *hist;     // [B][4096]
   uint32_t *hist2;    // [B][256]
-  uint32_t *ccount;   // [B]
-  uint32_t *flag;     // some row needs the tie refinement
   uint32_t *tiecnt;   // [B * per_row]
-  uint32_t *pair_done;  // [B * 2] item splits of (sequence, half) whose partials are written
+  uint32_t zone_hist_u4;  // the histograms' part of the zone, in 16-byte words
+  uint32_t *ccount;   // [B] candidates listed (only grows; each call reads its base first)
+  uint32_t *flag;     // the call's token when some row needs the tie refinement
+  uint32_t *pair_done;  // [B * 4] item splits of (sequence, quarter) whose partials are written (only grows)
   uint64_t *cand;     // [B][kCandCap]
-  float4 *ws_o;       // [B * 2 * S][64 column quads][128 heads] partial outputs
-  float2 *ws_ml;      // [B * 2 * S][128]                     (max, sum) in log2 units
+  float4 *ws_o;       // [B * 4 * S][32 column quads][128 heads] partial outputs
+  float2 *ws_ml;      // [B * 4 * S][128]                      (max, sum) in log2 units
 };
 
 struct StepArgs {
@@ -143,7 +158,7 @@ struct StepArgs {
   int64_t entry_cap;
   float sm_scale;
   int per_row;                  // scan CTAs per sequence
-  int S, cps;                   // item splits per (sequence, half) and chunks per split
+  int S, cps;                   // item splits per (sequence, quarter) and chunks per split
   int32_t *idx_out;
   float *score_out;
   __nv_bfloat16 *out;
@@ -313,7 +328,7 @@ __device__ __forceinline__ uint32_t block_scan_w(uint32_t v, Misc *misc, uint32_
 }
 
 // Warp-aggregated append of `key` (when take) to a global list with counter.
-__device__ __forceinline__ void list_append(bool take, uint64_t key, uint32_t *count, uint64_t *list) {
+__device__ __forceinline__ void list_append(bool take, uint64_t key, uint32_t *count, uint32_t cbase, uint64_t *list) {
   const int lane = threadIdx.x & 31;
   const unsigned msk = __ballot_sync(0xffffffffu, take);
   if (!msk) return;
@@ -322,7 +337,7 @@ __device__ __forceinline__ void list_append(bool take, uint64_t key, uint32_t *c
   if (lane == leader) base = atomicAdd(count, (uint32_t)__popc(msk));
   base = __shfl_sync(0xffffffffu, base, leader);
   if (take) {
-    const uint32_t pos = base + __popc(msk & ((1u << lane) - 1u));
+    const uint32_t pos = base - cbase + __popc(msk & ((1u << lane) - 1u));
     if (pos < (uint32_t)kCandCap) list[pos] = key;
   }
 }
@@ -384,10 +399,10 @@ __device__ __forceinline__ uint32_t quant4(const float (&C)[4], float s) {
 // ---------------------------------------------------------------------------
 // attention helpers
 // ---------------------------------------------------------------------------
-// Core-matrix layouts (8 rows x 16 B): KV [32 items][512 d] with g = d / 8,
-// g-stride 512 B and item-group stride 128 B; P [128 heads][32 items] with
-// g = item / 8, g-stride 2048 B and head-group stride 128 B.
-__device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 512 + (i >> 3) * 128 + (i & 7) * 16; }
+// Core-matrix layouts (8 rows x 16 B): the item tile KV [128 items][512 d]
+// with g = d / 8, g-stride 2 KiB and item-group stride 128 B; P [128 heads]
+// [128 items] with g = item / 8, g-stride 2 KiB and head-group stride 128 B.
+__device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 2048 + (i >> 3) * 128 + (i & 7) * 16; }
 __device__ __forceinline__ uint32_t p_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
 
 __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, uint4 &lo, uint4 &hi) {
@@ -408,52 +423,65 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, uint4 &lo, uint4
 
 __device__ __forceinline__ uint4 ldcg16(const void *p) { return __ldcg(reinterpret_cast<const uint4 *>(p)); }
 
-// Weighted sum of the item splits' partial outputs for tasks (head hh, column
-// quad c) of one unit: R tasks per thread, GJ splits per round, all R * GJ
-// loads in flight before any is used.  src: partials of split 0 offset to the
-// unit's first head ([split][64 quads][128 heads]); dst: output row of that
-// head at this half's first column.
-template <int R, int GJ>
-__device__ __forceinline__ void merge_tasks(const float4 *src, const float *wts, const float *inv_l, int S, int nh,
-                                            __nv_bfloat16 *dst) {
-  const int ntask = nh * 64;
-  for (int t0 = threadIdx.x; t0 < ntask; t0 += kThreads * R) {
-    float4 acc[R];
+// The same decision in every lane of the warp (after a bounded wait that may
+// give up in some lanes only), so that warp-collective TMEM loads and stores
+// and votes that follow are never reached by part of a warp.
+__device__ __forceinline__ bool uniform(bool v) { return __all_sync(0xffffffffu, v); }
+
+// 2^x (hardware approximation, a few ulp; flushes results below 2^-126 to 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Combines the S item splits' partials of heads [h0, h0 + nh) of one
+// (sequence, quarter).  One task per (head, column quad); each loads its
+// splits' (max, sum) and partial quad 8 at a time, all in flight, and folds
+// them into a running maximum, sum and accumulator.
+//   src_o: [S][32 quads][128 heads] float4,  src_ml: [S][128 heads],
+//   dst: the sequence's output at this quarter's first column,
+//   lse: the sequence's log-sum-exp row (or null).
+__device__ __forceinline__ void merge_quarter(const float4 *src_o, const float2 *src_ml, int S, int h0, int nh,
+                                              __nv_bfloat16 *dst, float *lse) {
+  const int ntask = nh * (DQ / 4);
+  for (int t = threadIdx.x; t < ntask; t += kThreads) {
+    const int h = h0 + t / (DQ / 4), c = t % (DQ / 4);
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < S; j0 += 8) {
+      float2 ml[8];
+      float4 v[8];
 #pragma unroll
-    for (int r = 0; r < R; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < S; j0 += GJ) {
-      float4 v[R][GJ];
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int t = t0 + r * kThreads;
-#pragma unroll
-        for (int jj = 0; jj < GJ; ++jj)
-          v[r][jj] = (t < ntask && j0 + jj < S) ? __ldcg(src + ((int64_t)(j0 + jj) * 64 + (t & 63)) * TH + (t >> 6))
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = j0 + jj;
+        ml[jj] = j < S ? __ldcg(src_ml + (int64_t)j * TH + h) : make_float2(-INFINITY, 0.f);
+        v[jj] = j < S ? __ldcg(src_o + ((int64_t)j * (DQ / 4) + c) * TH + h) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      float Mg = M;
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int t = t0 + r * kThreads;
+      for (int jj = 0; jj < 8; ++jj)
+        if (ml[jj].y > 0.f) Mg = fmaxf(Mg, ml[jj].x);
+      if (Mg == -INFINITY) continue;
+      const float f = M == -INFINITY ? 0.f : exp2f(M - Mg);
+      acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+      L *= f;
+      M = Mg;
 #pragma unroll
-        for (int jj = 0; jj < GJ; ++jj) {
-          const float wj = (t < ntask && j0 + jj < S) ? wts[(j0 + jj) * nh + (t >> 6)] : 0.f;
-          acc[r].x += wj * v[r][jj].x; acc[r].y += wj * v[r][jj].y;
-          acc[r].z += wj * v[r][jj].z; acc[r].w += wj * v[r][jj].w;
-        }
+      for (int jj = 0; jj < 8; ++jj) {
+        const float wj = ml[jj].y > 0.f ? exp2f(ml[jj].x - M) : 0.f;
+        L += wj * ml[jj].y;
+        acc.x += wj * v[jj].x; acc.y += wj * v[jj].y; acc.z += wj * v[jj].z; acc.w += wj * v[jj].w;
       }
     }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int t = t0 + r * kThreads;
-      if (t >= ntask) break;
-      const float il = inv_l[t >> 6];
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[r].x * il, acc[r].y * il);
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[r].z * il, acc[r].w * il);
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t *>(&lo);
-      pk.y = *reinterpret_cast<const uint32_t *>(&hi);
-      *reinterpret_cast<uint2 *>(dst + (int64_t)(t >> 6) * TD + (t & 63) * 4) = pk;
-    }
+    const float il = 1.f / L;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * il, acc.y * il);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * il, acc.w * il);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(dst + (int64_t)h * TD + c * 4) = pk;
+    if (lse && c == 0) lse[h] = (M + log2f(L)) * 0.6931471805599453f;
   }
 }
 
@@ -476,8 +504,11 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   const bool scanA = rowA < a.B;
   const int64_t tA = scanA ? (int64_t)a.q_pos[rowA] : -1;
   const int nvisA = tA < 0 ? 0 : (int)min((tA + 1) / a.m, (int64_t)a.n_entries);
-  const int slice = (nvisA + a.per_row - 1) / a.per_row;
-  const int s0 = min(part * slice, nvisA), s1 = min(s0 + slice, nvisA);
+  // contiguous key ranges; the last part, which also pools the new tokens,
+  // takes half a share: part p starts at 2 p nvis / (2 per_row - 1)
+  const int64_t den = 2 * (int64_t)a.per_row - 1;
+  const int s0 = (int)((2 * (int64_t)part * nvisA) / den);
+  const int s1 = part == a.per_row - 1 ? nvisA : (int)((2 * (int64_t)(part + 1) * nvisA) / den);
   const int n = s1 - s0;
   const int nb = (n + kBatchKeys - 1) / kBatchKeys;
   const int ybase = (int)((int64_t)rowA * a.entry_cap + s0);
@@ -487,6 +518,16 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   const int64_t e0 = e1 - nbn;
   const bool append_ok = tA >= 0 && (tA + 1) % a.m == 0 && e0 >= 0 && e1 <= a.entry_cap && tA + 1 >= a.n_new;
   if (scanA && part == 0 && tid == 0 && !append_ok) raise_status(a.status, STATUS_BAD_POSITION);
+
+  // the attention unit this CTA runs after the selection: (sequence, quarter
+  // of D, item split)
+  const int S = a.S;
+  const int units = a.B * 4 * S;
+  const bool attB = (int)blockIdx.x < units;
+  const int split = (int)blockIdx.x % S;
+  const int pair = (int)blockIdx.x / S;
+  const int qd = pair & 3;
+  const int rowB = min(pair >> 2, a.B - 1);
 
   uint64_t *full = bar + A_FULL;
   uint64_t *mdone = bar + A_MDONE;
@@ -499,11 +540,19 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       tc::tma_load_2d(kbuf + slot * kBatchBytes + i * 8192, &kmap, 0, ybase + bb * kBatchKeys + i * 256,
                       &full[slot]);
   };
-  if (tid == 0) gb_read_base(ws.bar, G, misc);
+  if (tid == 0) {
+    gb_read_base(ws.bar, G, misc);
+    // the unit's pair counter before any unit of this call adds to it (they
+    // do so only after the selection, which every CTA reaches after this)
+    if (attB) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(misc->pair_base) : "l"(ws.pair_done + pair) : "memory");
+    // the candidate counters grow during the selection, after every CTA read them here
+    if (scanA) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(misc->cbase_a) : "l"(ws.ccount + rowA) : "memory");
+    if (attB) asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(misc->cbase_b) : "l"(ws.ccount + rowB) : "memory");
+    misc->token = (uint32_t)(misc->base_ctr / G) + 1u;
+  }
   if (tid == kWork) {
     for (int i = 0; i < NBAR; ++i)
-      tc::mbar_init(&bar[i], (i == BAR_KV_FULL || i == BAR_KV_FULL + 1 || i == BAR_P_FULL || i == BAR_P_FULL + 1)
-                                 ? 128u : 1u);
+      tc::mbar_init(&bar[i], (i == BAR_KV_FULL || i == BAR_P_FULL || i == BAR_MX) ? 256u : i == BAR_QT ? 128u : 1u);
     misc->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     for (int bb = 0; bb < min(kStages, nb); ++bb) issue(bb);
@@ -533,17 +582,11 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         w16[h] = min(max(r, 0), 16);
       }
     }
-    // this CTA's share of the per-call counters
-    const uint32_t per = (ws.zone_u4 + G - 1) / G;
-    const uint32_t z0 = min(blockIdx.x * per, ws.zone_u4), z1 = min(z0 + per, ws.zone_u4);
-    uint4 *zp = reinterpret_cast<uint4 *>(ws.zone);
-    for (uint32_t i = z0 + tid; i < z1; i += kWork) zp[i] = make_uint4(0, 0, 0, 0);
   }
   tc::fence_proxy_async_smem();
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (tid == 0) gb_arrive(ws.bar, misc);            // barrier 0 (waited for after the scan)
   const uint32_t tbase = misc->tmem;
   if (warp < 4) {     // block scales 2^0 (UE8M0 127) wherever the MMA may read them
     const uint32_t ones[4] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
@@ -667,7 +710,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
     }
     if (bb > 0 && warp < 8) {
       const int pb = bb - 1;
-      const bool ok = bwait(&mdone[pb & 1], (uint32_t)(pb >> 1) & 1u, misc, a.status);
+      const bool ok = uniform(bwait(&mdone[pb & 1], (uint32_t)(pb >> 1) & 1u, misc, a.status));
       tc::fence_after_sync();
       const int q = warp & 3;
       uint32_t acc[4][4];
@@ -700,13 +743,6 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   }
 
   // ---------------------------------------------------------------- attention unit of this CTA
-  const int S = a.S;
-  const int units = a.B * 2 * S;
-  const bool attB = (int)blockIdx.x < units;
-  const int split = (int)blockIdx.x % S;
-  const int pair = (int)blockIdx.x / S;
-  const int dh = pair & 1;
-  const int rowB = min(pair >> 1, a.B - 1);
   int64_t tB = a.q_pos[rowB];
   if (tB < 0) tB = 0;
   const int nvisB = (int)min((tB + 1) / a.m, (int64_t)a.n_entries);
@@ -718,23 +754,14 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   const int c_begin = split * a.cps;
   const int c_end = min(c_begin + a.cps, nch);
   const int nloc = attB ? max(0, c_end - c_begin) : 0;
-  if (warp == 8 && attB) {
-    // the key ring is idle: Q for the attention, and the unit's window rows into L2
-    if (lane == 0 && nloc > 0) {
-      tc::mbar_arrive_expect_tx(&bar[BAR_Q], TH * TD * 2);
-      for (int k = 0; k < TD / 16; ++k)
-        tc::tma_load_2d(smem + B_Q + k * 4096, &qmap, 16 * k, rowB * TH, &bar[BAR_Q]);
-    }
-    const int u1 = min(c_end * CH, n_items);
-    for (int u = max(c_begin * CH, nsel) + lane; u < u1; u += 32) {
-      const uint8_t *src = a.wcodes + ((int64_t)rowB * a.win_cap + ((p0 + (u - nsel)) % a.win_cap)) * TD;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(TD) : "memory");
-    }
+  if (tid == kWork && nloc > 0) {
+    // the key ring is idle: Q of the unit's sequence in one 3-D TMA,
+    // [32 d-blocks][128 heads][16 d]
+    tc::mbar_arrive_expect_tx(&bar[BAR_Q], TH * TD * 2);
+    tc::tma_load_3d(smem + B_Q, &qmap, 0, rowB * TH, 0, &bar[BAR_Q]);
   }
 
   // ---------------------------------------------------------------- A2 select
-  if (tid == 0) gb_wait(ws.bar, G, misc, a.status);   // barrier 0: the counters are zero
-  __syncthreads();
   uint32_t *ghist = ws.hist + (int64_t)rowA * kBins;
   if (scanA && warp < 8) {
     for (int i = tid; i < kBins; i += kWork) {
@@ -764,7 +791,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       for (int j = tid; j < n; j += kWork) mine += (sc[j] >> 8) >= bstar ? 1u : 0u;
       uint32_t total;
       uint32_t pos = block_scan_w(mine, misc, &total);
-      if (tid == 0) misc->base = total ? atomicAdd(ccount, total) : 0u;
+      if (tid == 0) misc->base = total ? atomicAdd(ccount, total) - misc->cbase_a : 0u;
       wsync();
       pos += misc->base;
       for (int j = tid; j < n; j += kWork) {
@@ -780,7 +807,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         }
       }
     } else {
-      if (tid == 0 && part == 0) atomicOr(ws.flag, 1u);
+      if (tid == 0 && part == 0) atomicExch(ws.flag, misc->token);
       wsync();
       for (int i = tid; i < 256; i += kWork) hist[i] = 0;
       wsync();
@@ -795,7 +822,15 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   }
   grid_sync(ws.bar, G, misc, a.status);             // barrier 2: candidates listed
 
-  if (*(volatile uint32_t *)ws.flag) {               // the same decision in every CTA
+  // the same decision in every CTA; the histograms' last reads are done
+  const bool refine_any = *(volatile uint32_t *)ws.flag == misc->token;
+  if (warp < 8) {
+    const uint32_t per = (ws.zone_hist_u4 + G - 1) / G;
+    const uint32_t z0 = min(blockIdx.x * per, ws.zone_hist_u4), z1 = min(z0 + per, ws.zone_hist_u4);
+    uint4 *zp = reinterpret_cast<uint4 *>(ws.zone);
+    for (uint32_t i = z0 + tid; i < z1; i += kWork) zp[i] = make_uint4(0, 0, 0, 0);
+  }
+  if (refine_any) {
     uint32_t tstar = 0, take_ties = 0;
     if (scanA && refine && warp < 8) {
       if (tid == 0) {
@@ -817,7 +852,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       for (int j0 = 0; j0 < n; j0 += kWork) {
         const int j = j0 + tid;
         const uint32_t s = j < n ? sc[j] : 0u;
-        list_append(j < n && s > tstar, make_key(s, (uint32_t)(s0 + j)), ccount, cand);
+        list_append(j < n && s > tstar, make_key(s, (uint32_t)(s0 + j)), ccount, misc->cbase_a, cand);
         myties += (j < n && s == tstar) ? 1u : 0u;
       }
       myties = __reduce_add_sync(0xffffffffu, myties);
@@ -841,19 +876,28 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         const bool tie = j < n && sc[j] == tstar;
         const unsigned msk = __ballot_sync(0xffffffffu, tie);
         const uint32_t r = got + __popc(msk & ((1u << lane) - 1u));
-        list_append(tie && r < want, make_key(tstar, (uint32_t)(s0 + j)), ccount, cand);
+        list_append(tie && r < want, make_key(tstar, (uint32_t)(s0 + j)), ccount, misc->cbase_a, cand);
         got += __popc(msk);
       }
     }
     grid_sync(ws.bar, G, misc, a.status);           // barrier 4r: candidates listed
+    // the tie counters' last reads are done
+    if (warp < 8) {
+      const uint32_t nz = ws.zone_u4 - ws.zone_hist_u4;
+      const uint32_t per = (nz + G - 1) / G;
+      const uint32_t z0 = min(blockIdx.x * per, nz), z1 = min(z0 + per, nz);
+      uint4 *zp = reinterpret_cast<uint4 *>(ws.zone) + ws.zone_hist_u4;
+      for (uint32_t i = z0 + tid; i < z1; i += kWork) zp[i] = make_uint4(0, 0, 0, 0);
+    }
   }
 
-  // rank: each candidate's position is the number of larger keys
+  // rank: each candidate's position is the number of larger keys, counted
+  // by a warp; the row's CTAs share its candidates
   if (scanA && warp < 8) {
     const int cnt = min(a.K, nvisA);
     int32_t *oi = a.idx_out + (int64_t)rowA * a.K;
     float *os = a.score_out ? a.score_out + (int64_t)rowA * a.K : nullptr;
-    const uint32_t nc = min(__ldcg(ccount), (uint32_t)kCandCap);
+    const uint32_t nc = min(__ldcg(ccount) - misc->cbase_a, (uint32_t)kCandCap);
     uint64_t *ck = reinterpret_cast<uint64_t *>(smem + A_SC);   // the scores are no longer needed
     wsync();
     for (uint32_t i = tid; i < nc; i += kWork) ck[i] = __ldcg(cand + i);
@@ -884,83 +928,127 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   if (warp < 8)
     for (int i = tid; i < nsel_loc; i += kWork) sel[i] = __ldcg(a.idx_out + (int64_t)rowB * a.K + c_begin * CH + i);
   __syncthreads();
-  if (warp == 8 && nsel_loc > 0) {
-    for (int i = lane; i < nsel_loc; i += 32)
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.codes + ((int64_t)rowB * a.entry_cap + sel[i]) * TD),
-                   "r"(TD)
-                   : "memory");
-  }
   const uint32_t sbase = tc::smem_u32(smem);
   bool ok_b = true;
   float m_used = -INFINITY, l_sum = 0.f;
-  if (warp < 4) {
-    // ------------------------------------------------------------ loaders
-    const int i8 = lane & 7, pq = lane >> 3;
-    for (int lc = 0; lc < nloc; ++lc) {
-      const int buf = lc & 1;
-      const int item = warp * 8 + i8;
-      const int u = (c_begin + lc) * CH + item;
-      const uint8_t *src;
-      const float *scp;
-      if (u < nsel) {
-        const int64_t ent = (int64_t)rowB * a.entry_cap + sel[u - c_begin * CH];
-        src = a.codes + ent * TD;
-        scp = a.scales + ent;
-      } else {
-        // items past the list read a valid row (the first window token); their
-        // logits are masked and their P is zero
-        const int64_t p = p0 + (u < n_items ? u - nsel : 0);
-        const int64_t ent = (int64_t)rowB * a.win_cap + (p % a.win_cap);
-        src = a.wcodes + ent * TD;
-        scp = a.wscales + ent;
-      }
-      uint4 c[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) c[k] = ldcg16(src + 16 * (pq + 4 * k));
-      const float sc_raw = __ldcg(scp);
-      if (lc >= 2 && !bwait(&bar[BAR_KV_FREE + buf], ((lc - 2) >> 1) & 1, misc, a.status)) break;
-      const float scv = u < n_items ? sc_raw : 0.f;
-      unsigned char *kv = smem + B_KV + buf * KV_BYTES;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int p = pq + 4 * k;
-        uint4 lo, hi;
-        e4m3x16_to_bf16(c[k], lo, hi);
-        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p)) = lo;
-        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p + 1)) = hi;
-      }
-      if (pq == 0) iscale[buf * CH + item] = scv;
-      tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bar[BAR_KV_FULL + buf]);
-    }
-  } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax (one head per thread)
-    const int quad = warp - 4;
+  if (warp < 8) {
+    // ------------------------------------------------------------ workers
+    // Every worker gathers a share of each chunk; the softmax of a head runs
+    // on the two warps that own its TMEM lane (warp w and w + 4), each over
+    // half of the chunk's items; warps 4-7 also move Q into TMEM and run the
+    // epilogue.
+    const bool soft = warp >= 4;
+    const int quad = warp & 3;
+    const int half = soft ? 0 : 1;                    // items [64 half, 64 half + 64) of a chunk
+    const int h = quad * 32 + lane;                   // this thread's head (TMEM lane)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    float *mxx = reinterpret_cast<float *>(smem + B_MX);   // [2][128]
     const float qs = a.sm_scale * kLog2e;
     for (int c = 0; c < nloc && ok_b; ++c) {
-      const int buf = c & 1;
-      if (!bwait(&bar[BAR_KV_FULL + buf], (c >> 1) & 1, misc, a.status) ||
-          !bwait(&bar[BAR_S_FULL + buf], (c >> 1) & 1, misc, a.status)) { ok_b = false; break; }
-      tc::fence_after_sync();
-      uint32_t sr[32];
-      tc::tmem_ld32(tbase + lane_off + TCOL_S + buf * CH, sr);
-      tc::tmem_wait_ld();
-      const int valid = min(CH, n_items - (c_begin + c) * CH);
-      float s[32];
-      float mx = -INFINITY;
+      // gather: 4 threads per item row (8 x 16 B each), 2 rows per thread;
+      // the loads are issued before anything else waits
+      uint4 cv[2][8];
+      float scr[2];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        s[j] = (j < valid) ? __uint_as_float(sr[j]) * iscale[buf * CH + j] * qs : -INFINITY;
-        mx = fmaxf(mx, s[j]);
+      for (int r = 0; r < 2; ++r) {
+        const int t = tid + kWork * r;
+        const int item = t >> 2, pq = t & 3;
+        const int u = (c_begin + c) * CH + item;
+        const uint8_t *src;
+        const float *scp;
+        if (u < nsel) {
+          const int64_t ent = (int64_t)rowB * a.entry_cap + sel[u - c_begin * CH];
+          src = a.codes + ent * TD;
+          scp = a.scales + ent;
+        } else {
+          // items past the list read a valid row (the first window token);
+          // their logits are masked and their P is zero
+          const int64_t pp = p0 + (u < n_items ? u - nsel : 0);
+          const int64_t ent = (int64_t)rowB * a.win_cap + (pp % a.win_cap);
+          src = a.wcodes + ent * TD;
+          scp = a.wscales + ent;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) cv[r][k] = ldcg16(src + 16 * (pq + 4 * k));
+        scr[r] = u < n_items ? __ldcg(scp) : 0.f;
       }
+      if (c == 0) {
+        if (soft) {
+          // Q row h into TMEM while the gathers are in flight: d-block k of the
+          // staging buffer holds d = 16 k .. 16 k + 15; 32 TMEM columns take 4
+          // d-blocks (two bf16 per column)
+          const bool qok = uniform(bwait(&bar[BAR_Q], 0, misc, a.status));
+#pragma unroll 1
+          for (int cb = 0; cb < 8 && qok; ++cb) {
+            uint32_t v[32];
+#pragma unroll
+            for (int db = 0; db < 4; ++db) {
+              const uint4 *q4 = reinterpret_cast<const uint4 *>(smem + B_Q + ((cb * 4 + db) * TH + h) * 32);
+              const uint4 x0 = q4[0], x1 = q4[1];
+              v[db * 8 + 0] = x0.x; v[db * 8 + 1] = x0.y; v[db * 8 + 2] = x0.z; v[db * 8 + 3] = x0.w;
+              v[db * 8 + 4] = x1.x; v[db * 8 + 5] = x1.y; v[db * 8 + 6] = x1.z; v[db * 8 + 7] = x1.w;
+            }
+            tc::tmem_st32(tbase + lane_off + TCOL_Q + cb * 32, v);
+          }
+          tc::tmem_wait_st();
+          tc::fence_before_sync();
+          tc::mbar_arrive(&bar[BAR_QT]);
+          if (!qok) ok_b = false;
+        }
+        // the tile overlays the Q staging buffer: every head must be copied
+        if (!uniform(bwait(&bar[BAR_QT], 0, misc, a.status) && ok_b)) { ok_b = false; break; }
+      } else if (!uniform(bwait(&bar[BAR_KV_FREE], (c - 1) & 1, misc, a.status))) {
+        ok_b = false;
+        break;
+      }
+      unsigned char *kv = smem + B_KV;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int t = tid + kWork * r;
+        const int item = t >> 2, pq = t & 3;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int pc = pq + 4 * k;
+          uint4 lo, hi;
+          e4m3x16_to_bf16(cv[r][k], lo, hi);
+          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * pc)) = lo;
+          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * pc + 1)) = hi;
+        }
+        if (pq == 0) iscale[item] = scr[r];
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bar[BAR_KV_FULL]);
+      // -------------------------------------------------------- softmax of chunk c
+      if (!uniform(bwait(&bar[BAR_S_FULL], c & 1, misc, a.status))) { ok_b = false; break; }
+      tc::fence_after_sync();
+      const int valid = min(CH, n_items - (c_begin + c) * CH);
+      const int i_lo = half * (CH / 2);
+      float pmx = -INFINITY;
+#pragma unroll 1
+      for (int jb = 0; jb < CH / 64; ++jb) {
+        uint32_t sr[32];
+        tc::tmem_ld32(tbase + lane_off + TCOL_S + i_lo + jb * 32, sr);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int i = i_lo + jb * 32 + j;
+          if (i < valid) pmx = fmaxf(pmx, __uint_as_float(sr[j]) * iscale[i] * qs);
+        }
+      }
+      // the two halves agree on the chunk maximum through shared memory
+      mxx[half * TH + h] = pmx;
+      tc::mbar_arrive(&bar[BAR_MX]);
+      if (!uniform(bwait(&bar[BAR_MX], c & 1, misc, a.status))) { ok_b = false; break; }
+      const float mx = fmaxf(mxx[h], mxx[TH + h]);
       const bool need = mx > m_used + kRescaleLog2;
       if (c > 0 && __any_sync(0xffffffffu, need)) {
-        if (!bwait(&bar[BAR_PV_DONE], (c - 1) & 1, misc, a.status)) { ok_b = false; break; }
+        // O holds earlier chunks: wait for the last PV, then rescale this
+        // warp's half of the head rows' quarter (2 of 4 column blocks)
+        if (!uniform(bwait(&bar[BAR_PV_DONE], (c - 1) & 1, misc, a.status))) { ok_b = false; break; }
         tc::fence_after_sync();
-        const float f = need ? exp2f(m_used - mx) : 1.f;
+        const float f = need ? ex2(m_used - mx) : 1.f;
 #pragma unroll 1
-        for (int blk = 0; blk < DHALF / 32; ++blk) {
+        for (int blk = 2 * half; blk < 2 * half + 2; ++blk) {
           uint32_t o[32];
           tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
           tc::tmem_wait_ld();
@@ -971,120 +1059,126 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         tc::tmem_wait_st();
       }
       if (need) {
-        l_sum = (m_used == -INFINITY) ? 0.f : l_sum * exp2f(m_used - mx);
+        l_sum = (m_used == -INFINITY) ? 0.f : l_sum * ex2(m_used - mx);
         m_used = mx;
       }
-      uint32_t pw[16];
+      // P = p * item scale (bf16) for this half's items, in the core-matrix
+      // layout of the PV A operand
+      unsigned char *P = smem + B_P;
       float lsum = 0.f;
+#pragma unroll 1
+      for (int jb = 0; jb < CH / 64; ++jb) {
+        uint32_t sr[32];
+        tc::tmem_ld32(tbase + lane_off + TCOL_S + i_lo + jb * 32, sr);
+        tc::tmem_wait_ld();
+        uint32_t pw[16];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float pa = exp2f(s[j] - m_used), pb = exp2f(s[j + 1] - m_used);
-        lsum += pa + pb;
-        const __nv_bfloat162 v = __floats2bfloat162_rn(pa * iscale[buf * CH + j], pb * iscale[buf * CH + j + 1]);
-        pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+        for (int j = 0; j < 32; j += 2) {
+          const int i0 = i_lo + jb * 32 + j;
+          const float sa = i0 < valid ? __uint_as_float(sr[j]) * iscale[i0] * qs : -INFINITY;
+          const float sb = i0 + 1 < valid ? __uint_as_float(sr[j + 1]) * iscale[i0 + 1] * qs : -INFINITY;
+          const float pa = ex2(sa - m_used), pb = ex2(sb - m_used);
+          lsum += pa + pb;
+          const __nv_bfloat162 v = __floats2bfloat162_rn(pa * iscale[i0], pb * iscale[i0 + 1]);
+          pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+        }
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg)
+          *reinterpret_cast<uint4 *>(P + p_off(h, (i_lo + jb * 32) / 8 + gg)) =
+              make_uint4(pw[4 * gg], pw[4 * gg + 1], pw[4 * gg + 2], pw[4 * gg + 3]);
       }
       l_sum += lsum;
-      unsigned char *P = smem + B_P + buf * P_BYTES;
-      const int h = quad * 32 + lane;
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        *reinterpret_cast<uint4 *>(P + p_off(h, g)) = make_uint4(pw[4 * g], pw[4 * g + 1], pw[4 * g + 2], pw[4 * g + 3]);
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
-      tc::mbar_arrive(&bar[BAR_P_FULL + buf]);
+      tc::mbar_arrive(&bar[BAR_P_FULL]);
     }
-    // epilogue: the normalised half row (one split) or the unnormalised partial
-    const int h = quad * 32 + lane;
-    const int64_t orow = (int64_t)rowB * TH + h;
-    const bool have = nloc > 0 && ok_b && bwait(&bar[BAR_PV_DONE], (nloc - 1) & 1, misc, a.status);
-    tc::fence_after_sync();
-    if (attB && S == 1) {
-      if (have) {
-        const float inv = 1.f / l_sum;
-#pragma unroll 1
-        for (int blk = 0; blk < DHALF / 32; ++blk) {
-          uint32_t o[32];
-          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
-          tc::tmem_wait_ld();
-          uint32_t wv[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv);
-            wv[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * TD + dh * DHALF + blk * 32);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
-        }
-        if (a.lse && dh == 0) a.lse[orow] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
-      }
-    } else if (attB) {
-      // the unnormalised partial as [64 column quads][128 heads] float4 (a
-      // warp's store covers 512 contiguous bytes), then (max, sum); each
-      // writer makes its stores visible before the unit is counted done
-      const int64_t slot = (int64_t)pair * S + split;
-      float4 *dst = ws.ws_o + slot * 64 * TH + h;
-#pragma unroll 1
-      for (int blk = 0; blk < DHALF / 32; ++blk) {
-        uint32_t o[32];
+    // the row sums of the two halves (every worker arrives here, whatever
+    // happened in the loop)
+    asm volatile("bar.sync 6, 256;" ::: "memory");
+    mxx[half * TH + h] = l_sum;
+    asm volatile("bar.sync 6, 256;" ::: "memory");
+    if (soft) {
+      l_sum = mxx[h] + mxx[TH + h];
+      // epilogue: the normalised quarter row (one split) or the unnormalised
+      // partial.  FIN completes once, after every MMA of the CTA.
+      const int64_t orow = (int64_t)rowB * TH + h;
+      const bool have = uniform(nloc > 0 && ok_b && bwait(&bar[BAR_FIN], 0, misc, a.status));
+      tc::fence_after_sync();
+      if (attB && S == 1) {
         if (have) {
-          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
-          tc::tmem_wait_ld();
-        } else {
+          const float inv = 1.f / l_sum;
+#pragma unroll 1
+          for (int blk = 0; blk < DQ / 32; ++blk) {
+            uint32_t o[32];
+            tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
+            tc::tmem_wait_ld();
+            uint32_t wv[16];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
+            for (int j = 0; j < 32; j += 2) {
+              const __nv_bfloat162 v =
+                  __floats2bfloat162_rn(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv);
+              wv[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * TD + qd * DQ + blk * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
+          }
+          if (a.lse && qd == 0) a.lse[orow] = (m_used + log2f(l_sum)) * 0.6931471805599453f;
         }
+      } else if (attB) {
+        // the unnormalised partial as [32 column quads][128 heads] float4 (a
+        // warp's store covers 512 contiguous bytes), then (max, sum); each
+        // writer makes its stores visible before the unit is counted done
+        const int64_t slot = (int64_t)pair * S + split;
+        float4 *dst = ws.ws_o + slot * (DQ / 4) * TH + h;
+#pragma unroll 1
+        for (int blk = 0; blk < DQ / 32; ++blk) {
+          uint32_t o[32];
+          if (have) {
+            tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
+            tc::tmem_wait_ld();
+          } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          dst[(blk * 8 + k) * TH] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                                __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[(blk * 8 + k) * TH] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                                                  __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+        }
+        ws.ws_ml[slot * TH + h] = have ? make_float2(m_used, l_sum) : make_float2(-INFINITY, 0.f);
+        __threadfence();
+        asm volatile("bar.sync 4, 128;" ::: "memory");
+        if (h == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ws.pair_done + pair) : "memory");
       }
-      ws.ws_ml[slot * TH + h] = have ? make_float2(m_used, l_sum) : make_float2(-INFINITY, 0.f);
-      __threadfence();
-      asm volatile("bar.sync 4, 128;" ::: "memory");
-      if (h == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ws.pair_done + pair) : "memory");
     }
   } else {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nloc > 0) {
       const uint32_t idesc_qk = tc::idesc_bf16_f32(128, CH, 0, 0);
-      const uint32_t idesc_pv = tc::idesc_bf16_f32(128, DHALF, 0, 1);
-      auto issue_qk = [&](int c) {
-        const int buf = c & 1;
-        const uint32_t kvb = sbase + B_KV + buf * KV_BYTES;
-#pragma unroll 4
-        for (int k = 0; k < TD / 16; ++k) {
-          const uint64_t ad = tc::smem_desc_sw32(sbase + B_Q + k * 4096);
-          const uint64_t bd = tc::smem_desc(kvb + k * 1024, 512, 128);
-          tc::mma_bf16_ss(tbase + TCOL_S + buf * CH, ad, bd, idesc_qk, k > 0);
-        }
-        tc::mma_commit(&bar[BAR_S_FULL + buf]);
-      };
-      bool ok = bwait(&bar[BAR_Q], 0, misc, a.status) && bwait(&bar[BAR_KV_FULL + 0], 0, misc, a.status);
-      if (ok) { tc::fence_after_sync(); issue_qk(0); }
-      if (ok && nloc > 1) {
-        ok = bwait(&bar[BAR_KV_FULL + 1], 0, misc, a.status);
-        if (ok) { tc::fence_after_sync(); issue_qk(1); }
-      }
+      const uint32_t idesc_pv = tc::idesc_bf16_f32(128, DQ, 0, 1);
+      bool ok = bwait(&bar[BAR_QT], 0, misc, a.status);
       for (int c = 0; c < nloc && ok; ++c) {
-        const int buf = c & 1;
-        if (!bwait(&bar[BAR_P_FULL + buf], (c >> 1) & 1, misc, a.status)) break;
+        if (!bwait(&bar[BAR_KV_FULL], c & 1, misc, a.status)) break;
         tc::fence_after_sync();
-        const uint32_t pb = sbase + B_P + buf * P_BYTES;
-        const uint32_t vb = sbase + B_KV + buf * KV_BYTES + dh * (DHALF / 8) * 512;
+        // S = Q K^T: A = Q from TMEM (8 columns per K step of 16 d), B = the
+        // item tile, K-major core matrices (LBO = d-group step, SBO = 8 items)
+#pragma unroll 4
+        for (int k = 0; k < TD / 16; ++k)
+          tc::mma_bf16_ts(tbase + TCOL_S, tbase + TCOL_Q + 8 * k, tc::smem_desc(sbase + B_KV + k * 4096, 2048, 128),
+                          idesc_qk, k > 0);
+        tc::mma_commit(&bar[BAR_S_FULL]);
+        if (!bwait(&bar[BAR_P_FULL], c & 1, misc, a.status)) break;
+        tc::fence_after_sync();
+        // O += P V: A = P (K-major, K = items), B = the item tile read MN-major
+        // for this quarter of D (LBO = item-group step, SBO = d-group step)
+        const uint32_t vb = sbase + B_KV + qd * (DQ / 8) * 2048;
 #pragma unroll
-        for (int kk = 0; kk < CH / 16; ++kk) {
-          const uint64_t ad = tc::smem_desc(pb + kk * 4096, 2048, 128);
-          const uint64_t bd = tc::smem_desc(vb + kk * 256, 128, 512);
-          tc::mma_bf16_ss(tbase + TCOL_O, ad, bd, idesc_pv, (c > 0 || kk > 0));
-        }
-        tc::mma_commit(&bar[BAR_KV_FREE + buf]);
+        for (int kk = 0; kk < CH / 16; ++kk)
+          tc::mma_bf16_ss(tbase + TCOL_O, tc::smem_desc(sbase + B_P + kk * 4096, 2048, 128),
+                          tc::smem_desc(vb + kk * 256, 128, 2048), idesc_pv, (c > 0 || kk > 0));
+        tc::mma_commit(&bar[BAR_KV_FREE]);
         tc::mma_commit(&bar[BAR_PV_DONE]);
-        if (c + 2 < nloc) {
-          if (!bwait(&bar[BAR_KV_FULL + buf], ((c + 2) >> 1) & 1, misc, a.status)) break;
-          tc::fence_after_sync();
-          issue_qk(c + 2);
-        }
       }
       tc::mma_commit(&bar[BAR_FIN]);
       bwait(&bar[BAR_FIN], 0, misc, a.status);
@@ -1093,16 +1187,17 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
   }
 
   // ---------------------------------------------------------------- merge of the item splits
-  // Each unit combines heads [h0, h1) of its (sequence, half) once all S
+  // Each unit combines heads [h0, h1) of its (sequence, quarter) once all S
   // partials of that pair are counted:
   //   out = sum_j 2^(m_j - M) O_j / sum_j 2^(m_j - M) l_j,  M = max_j m_j.
   if (S > 1 && attB) {
     if (tid == 0 && !misc->abort) {
+      const uint32_t target = misc->pair_base + (uint32_t)S;
       const uint64_t t0 = gtimer();
       uint32_t v, it = 0;
       for (;;) {
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ws.pair_done + pair) : "memory");
-        if (v >= (uint32_t)S) break;
+        if ((int32_t)(v - target) >= 0) break;
         if ((++it & 63u) == 0 && gtimer() - t0 > kWaitNs) {
           misc->abort = 1;
           raise_status(a.status, STATUS_TIMEOUT);
@@ -1112,35 +1207,10 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       __threadfence();
     }
     __syncthreads();
-    const int h0 = split * TH / S, h1 = (split + 1) * TH / S, nh = h1 - h0;
+    const int h0 = split * TH / S, h1 = (split + 1) * TH / S;
     const int64_t slot0 = (int64_t)pair * S;
-    float *wts = reinterpret_cast<float *>(smem + B_P);        // [S][nh] split weights, then [nh] 1/L
-    float *inv_l = wts + S * nh;
-    float2 *mls = reinterpret_cast<float2 *>(smem + B_KV);     // [S][nh]
-    for (int i = tid; i < S * nh; i += kThreads) {
-      const int j = i / nh, hh = i - j * nh;
-      mls[i] = __ldcg(ws.ws_ml + (slot0 + j) * TH + h0 + hh);
-    }
-    __syncthreads();
-    for (int hh = tid; hh < nh; hh += kThreads) {
-      float M = -INFINITY;
-      for (int j = 0; j < S; ++j)
-        if (mls[j * nh + hh].y > 0.f) M = fmaxf(M, mls[j * nh + hh].x);
-      float L = 0.f;
-      for (int j = 0; j < S; ++j) {
-        const float2 ml = mls[j * nh + hh];
-        const float wj = ml.y > 0.f ? exp2f(ml.x - M) : 0.f;
-        wts[j * nh + hh] = wj;
-        L += wj * ml.y;
-      }
-      inv_l[hh] = 1.f / L;
-      if (a.lse && dh == 0) a.lse[(int64_t)rowB * TH + h0 + hh] = (M + log2f(L)) * 0.6931471805599453f;
-    }
-    __syncthreads();
-    const float4 *src = ws.ws_o + slot0 * 64 * TH + h0;
-    __nv_bfloat16 *dst = a.out + ((int64_t)rowB * TH + h0) * TD + dh * DHALF;
-    if (S <= 4) merge_tasks<4, 4>(src, wts, inv_l, S, nh, dst);
-    else merge_tasks<1, 16>(src, wts, inv_l, S, nh, dst);
+    merge_quarter(ws.ws_o + slot0 * (DQ / 4) * TH, ws.ws_ml + slot0 * TH, S, h0, h1 - h0,
+                  a.out + (int64_t)rowB * TH * TD + qd * DQ, (a.lse && qd == 0) ? a.lse + (int64_t)rowB * TH : nullptr);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -1182,14 +1252,14 @@ bool ds_plan(const csa_dims *d, int n_new, Plan *p) {
                 n_new, d->m, kMaxNew), false;
   const int G = ds_sms();
   if (G < 1) return fail(CSA_ERR_CUDA, "csa_decode_step: cannot size the grid (no device?)"), false;
-  if (d->B < 1 || 2 * d->B > G)
-    return fail(CSA_ERR_UNSUPPORTED, "csa_decode_step: B=%d (1..%d sequences)", d->B, G / 2), false;
+  if (d->B < 1 || 4 * d->B > G)
+    return fail(CSA_ERR_UNSUPPORTED, "csa_decode_step: B=%d (1..%d sequences)", d->B, G / 4), false;
   const int per_row = G / d->B;
-  if ((d->n_entries + per_row - 1) / per_row > kLocalCap)
+  if ((2 * (int64_t)d->n_entries + 2 * per_row - 2) / (2 * per_row - 1) + 1 > kLocalCap)
     return fail(CSA_ERR_UNSUPPORTED, "csa_decode_step: %d entries over %d CTAs per sequence (at most %d each)",
                 d->n_entries, per_row, kLocalCap), false;
   const int nch = (d->K + d->W + CH - 1) / CH;
-  int S = min(G / (2 * d->B), nch);
+  int S = min(min(G / (4 * d->B), nch), kMaxSplits);
   const int cps = (nch + S - 1) / S;
   S = (nch + cps - 1) / cps;
   if (cps * CH > kMaxSelLocal)
@@ -1209,22 +1279,24 @@ size_t ds_workspace(const csa_dims *d, const Plan &p, Ws *ws, void *base) {
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off += (bytes + 255) & ~(size_t)255; return o; };
   const size_t o_bar = take(8);
-  const size_t o_hist = take((size_t)(B * kBins * 4));
-  const size_t o_hist2 = take((size_t)(B * 256 * 4));
   const size_t o_cnt = take((size_t)(B * 4));
   const size_t o_flag = take(4);
+  const size_t o_hist = take((size_t)(B * kBins * 4));
+  const size_t hist_end = off;
+  const size_t o_hist2 = take((size_t)(B * 256 * 4));
   const size_t o_tie = take((size_t)(B * p.per_row * 4));
-  const size_t o_pair = take((size_t)(B * 2 * 4));
   const size_t zone_end = off;
+  const size_t o_pair = take((size_t)(B * 4 * 4));
   const size_t o_cand = take((size_t)(B * kCandCap * 8));
-  const int64_t slots = p.S > 1 ? B * 2 * p.S : 0;
-  const size_t o_o = take((size_t)(slots * TH * DHALF * 4));
+  const int64_t slots = p.S > 1 ? B * 4 * p.S : 0;
+  const size_t o_o = take((size_t)(slots * TH * DQ * 4));
   const size_t o_ml = take((size_t)(slots * TH * 8));
   if (ws && base) {
     char *c = static_cast<char *>(base);
     ws->bar = reinterpret_cast<unsigned long long *>(c + o_bar);
     ws->zone = reinterpret_cast<uint32_t *>(c + o_hist);
     ws->zone_u4 = (uint32_t)((zone_end - o_hist) / 16);
+    ws->zone_hist_u4 = (uint32_t)((hist_end - o_hist) / 16);
     ws->hist = reinterpret_cast<uint32_t *>(c + o_hist);
     ws->hist2 = reinterpret_cast<uint32_t *>(c + o_hist2);
     ws->ccount = reinterpret_cast<uint32_t *>(c + o_cnt);
@@ -1270,8 +1342,12 @@ int launch_decode_step(const float *x_new, const float *z_new, int n_new, const 
   if (!encode_tmap_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, kI, 32, (uint64_t)d->B * d->entry_cap, 32, 32, 256,
                       CU_TENSOR_MAP_SWIZZLE_32B))
     return fail(CSA_ERR_INVALID, "csa_decode_step: cannot map the indexer keys for TMA");
-  if (!encode_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, TD, (uint64_t)d->B * TH, TD * 2, 16, TH,
-                      CU_TENSOR_MAP_SWIZZLE_32B))
+  // Q as [32 d-blocks][B * 128 rows][16 d]: one box of 16 x 128 x 32 lands as
+  // [d-block][head][16 d] in shared memory
+  const uint64_t qdims[3] = {16, (uint64_t)d->B * TH, TD / 16};
+  const uint64_t qstrides[2] = {TD * 2, 32};
+  const uint32_t qbox[3] = {16, TH, TD / 16};
+  if (!encode_tmap_3d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, qdims, qstrides, qbox))
     return fail(CSA_ERR_INVALID, "csa_decode_step: cannot map the queries for TMA");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.G);

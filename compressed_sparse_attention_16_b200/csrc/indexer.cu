@@ -1216,7 +1216,8 @@ index_decode_kernel(const __grid_constant__ CUtensorMap kmap, const uint8_t *__r
     }
     if (bb > 0) {
       const int pb = bb - 1;
-      const bool ok = bwait(&mdone[pb & 1], (uint32_t)(pb >> 1) & 1u);
+      // one decision per warp: the TMEM loads below are warp-collective
+      const bool ok = __all_sync(0xffffffffu, bwait(&mdone[pb & 1], (uint32_t)(pb >> 1) & 1u));
       tc::fence_after_sync();
       // the key slot of batch pb is free again
       if (tid == 0 && pb + kFdStages < nb) issue(pb + kFdStages);

@@ -257,14 +257,14 @@ int hca_attend(const uint16_t *q, const uint8_t *codes, const float *scales,
  *   idx_out int32 [B, 1, K];  score_out fp32 [B, 1, K] or NULL
  *   out bf16 [B, 1, H, D];  lse fp32 [B, 1, H] or NULL
  *   workspace     at least csa_decode_step_workspace(d, n_new) bytes.  It must
- *                 be zero-filled once before its first use (cudaMemset after
- *                 allocation); every call leaves the words that carry its grid
- *                 barriers in the state the next call expects, and zeroes its
- *                 own counters.  After a call that timed out (csa_sync_status
- *                 returns CSA_ERR_TIMEOUT) zero it again.  Calls that share a
- *                 workspace must not overlap on the GPU.
+ *                 be zero-filled before its first use (cudaMemset after
+ *                 allocation); every call then leaves it in the state the next
+ *                 call with the same shape expects.  Zero it again when B, K,
+ *                 W or the GPU changes, and after a call that timed out
+ *                 (csa_sync_status returns CSA_ERR_TIMEOUT).  Calls that share
+ *                 a workspace must not overlap on the GPU.
  * Supported: H = 128, D = 512, dI = 64, HI <= 4, Tq = 1, K <= 2048, n_new a
- * multiple of m with n_new <= 16 and n_new <= win_cap, 2*B <= the GPU's SM
+ * multiple of m with n_new <= 16 and n_new <= win_cap, 4*B <= the GPU's SM
  * count, at most 8,192 visible entries per CTA (B sequences share the SMs).
  * Anything else returns CSA_ERR_UNSUPPORTED before any launch (use the
  * separate calls); csa_decode_step_workspace returns 0 for such shapes.
