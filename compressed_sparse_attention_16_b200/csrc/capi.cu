@@ -264,7 +264,7 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
   if (int rc = check_index_dims("csa_index_topk", d)) return rc;
   if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
   if (!qI || !w || !kI || !q_pos || !idx_out) return fail(CSA_ERR_INVALID, "csa_index_topk: NULL buffer");
-  if (!aligned16(kI) || ((uintptr_t)qI & 3) || ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) ||
+  if (!aligned16(kI) || !aligned16(qI) || ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) ||
       ((uintptr_t)idx_out & 3) || ((uintptr_t)score_out & 3))
     return fail(CSA_ERR_INVALID, "csa_index_topk: misaligned buffer");
   const size_t need = index_topk_workspace(d);

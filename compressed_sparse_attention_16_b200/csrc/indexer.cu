@@ -1803,6 +1803,11 @@ int launch_prefill_tc(const uint8_t *qI, const float *w, const uint8_t *kI, cons
 
 }  // namespace
 
+bool prefill2_plan(const csa_dims *d);
+size_t prefill2_workspace(const csa_dims *d);
+int launch_prefill2(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos, const csa_dims *d,
+                    int32_t *idx_out, float *score_out, void *workspace, cudaStream_t stream);
+
 size_t index_topk_workspace(const csa_dims *d) {
   int splits, slice, per_row;
   if (fd_plan(d, &per_row)) {
@@ -1812,6 +1817,7 @@ size_t index_topk_workspace(const csa_dims *d) {
     return a > b ? a : b;
   }
   if (tc_plan(d, &splits, &slice)) return tc_workspace(d, nullptr, nullptr);
+  if (prefill2_plan(d)) return prefill2_workspace(d);
   if (prefill_tc_plan(d)) return (size_t)((int64_t)d->B * d->Tq * d->K * 4);
   if (split_plan(d, &splits, &slice)) return (size_t)((int64_t)d->B * d->Tq * splits * d->K * 8);
   const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
@@ -1832,6 +1838,7 @@ int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, cons
   }
   if (tc_plan(d, &splits, &slice))
     return launch_tc(qI, w, kI, q_pos, d, splits, slice, idx_out, score_out, workspace, stream);
+  if (prefill2_plan(d)) return launch_prefill2(qI, w, kI, q_pos, d, idx_out, score_out, workspace, stream);
   if (prefill_tc_plan(d)) return launch_prefill_tc(qI, w, kI, q_pos, d, idx_out, score_out, workspace, stream);
   if (split_plan(d, &splits, &slice)) {
     uint64_t *cand = static_cast<uint64_t *>(workspace);

@@ -134,7 +134,7 @@ int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D
  * lists the min(K, n_vis) best entries in rank order -- score descending, ties
  * to the lower index -- followed by -1 padding.
  *
- *   qI         u8   [B, Tq, HI, dI/2]   packed E2M1
+ *   qI         u8   [B, Tq, HI, dI/2]   packed E2M1, 16-byte aligned
  *   w          fp32 [B, Tq, HI]
  *   kI         u8   [B, entry_cap, dI/2] packed E2M1
  *   q_pos      int32 [B, Tq]             (>= 0)
@@ -164,8 +164,8 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
  * shape takes: up to 64 query rows with >= 2,048 entries, 4 bytes per
  * (row, entry) plus 32 KiB per row (16 rows x 16,384 entries: 1.5 MiB;
  * 64 rows x 20,000 entries: 7.2 MiB); 65 to 148 decode rows, about 33 KiB
- * per row; the prefill path (> 64 rows, <= 65,535 entries), 4 bytes per
- * (row, K), i.e. up to 4,096 rows at K = 512.  The library allocates nothing
+ * per row; the prefill path (> 64 rows, K <= 1,024), 16 bytes per
+ * (row, K), i.e. up to 1,023 rows at K = 512.  The library allocates nothing
  * and calls no allocating routine.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any

@@ -184,3 +184,31 @@ def test_split_merge_path(HI, dI):
     pos = torch.randint(0, 4 * N + 10, (B, Tq), generator=g, dtype=torch.int32)
     pos[0, :4] = torch.tensor([1, 4 * 512 - 1, 4 * 512 + 3, 4 * N - 1], dtype=torch.int32)
     _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
+
+
+@pytest.mark.parametrize("K", [1, 37, 1024])
+def test_prefill_streaming_path_k_range(K):
+    """The >64-row streaming selection at the extremes of its k range, three
+    sequences of a length that is not a multiple of the 128-query block, with
+    rows below, at and above k visible entries."""
+    B, Tq, N, m = 3, 333, 4100, 4
+    inp = synth.indexer_inputs(B, Tq, N, 4, 64, seed=40 + K)
+    g = torch.Generator().manual_seed(K)
+    pos = torch.randint(0, 4 * N + 10, (B, Tq), generator=g, dtype=torch.int32)
+    pos[0, :6] = torch.tensor([0, 3, 4 * K - 1, 4 * K, 4 * K + 3, 4 * N - 1], dtype=torch.int32)
+    _compare(inp.qI, inp.w, inp.kI, pos, m, K, N)
+
+
+def test_prefill_streaming_path_crowded_bins():
+    """Keys drawn from a few codes give scores with few distinct values: the
+    threshold bin overflows the candidate buffer, so the finer histogram
+    levels run, down to exact ties taken in index order; one sequence has
+    identical keys (every score equal)."""
+    g = torch.Generator().manual_seed(9)
+    B, Tq, N, m, K = 2, 200, 5000, 4, 300
+    codes = torch.randint(0, 3, (B, N, 64), generator=g, dtype=torch.uint8)
+    codes[1] = 2
+    kI = (codes[..., 0::2] | (codes[..., 1::2] << 4)).contiguous()
+    inp = synth.indexer_inputs(B, Tq, 1, 4, 64, seed=41)
+    pos = torch.randint(4 * K, 4 * N + 40, (B, Tq), generator=g, dtype=torch.int32)
+    _compare(inp.qI, inp.w, kI, pos, m, K, N)
