@@ -466,7 +466,7 @@ index_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const uint8_t *__
         const bool ok = __all_sync(0xffffffffu, bwait(&tfull[grp], (uint32_t)use & 1u));
         tc::fence_after_sync();
         uint32_t r[4][16];
-#pragma unroll 1
+#pragma unroll
         for (int c = 0; c < kN / 16 - 1; ++c) {
           tmem_ld_heads16<HI>(taddr0 + c * 16, r);
           tc::tmem_wait_ld();
