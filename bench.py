@@ -432,7 +432,12 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     import torch
     import torch.distributed as dist
 
-    r = Runner(wl, seed=rank, device=dev, fused=args.decode_path == "fused")
+    if args.decode_path == "auto":
+        from compressed_sparse_attention_16_b200.pipeline import prefer_fused_step
+        fused = prefer_fused_step(wl.B, dev)
+    else:
+        fused = args.decode_path == "fused"
+    r = Runner(wl, seed=rank, device=dev, fused=fused)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     use_graph = r.decode and not args.no_graph
 
@@ -683,6 +688,8 @@ KERNEL_SOURCES = {
     "attend_tc_kernel": ["attend_tc.cu"],
     "attend_prefill_kernel": ["attend_prefill.cu"],
     "index_decode_kernel<4>": ["indexer.cu"],
+    "index_prefill_kernel<4>": ["index_prefill.cu"],
+    "decode_step_kernel<4>": ["decode_step.cu"],
 }
 SHARED_SOURCES = ["common.cuh", "tc.cuh"]
 
@@ -966,9 +973,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch decode steps without CUDA graphs")
-    ap.add_argument("--decode-path", default="fused", choices=["separate", "fused"],
-                    help="CSA decode steps as the separate calls (compress, index_topk, attend) or as one "
-                         "csa_decode_step launch")
+    ap.add_argument("--decode-path", default="auto", choices=["auto", "separate", "fused"],
+                    help="CSA decode steps as the separate calls (compress, index_topk, attend), as one "
+                         "csa_decode_step launch, or (auto) whichever pipeline.prefer_fused_step picks")
     ap.add_argument("--rows", type=int, default=0, help="kernel-case: query rows of a prefill workload")
     ap.add_argument("--kernel-case", default=None,
                     help="run one library call (index_topk, attend, hca_attend, compress_entry, "

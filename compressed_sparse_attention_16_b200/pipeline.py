@@ -23,6 +23,16 @@ from . import (Dims, attend, attend_workspace, compress, decode_step, decode_ste
                index_topk_workspace)
 
 
+def prefer_fused_step(B: int, device=None) -> bool:
+    """Whether one csa_decode_step launch beats the separate calls for B
+    sequences.  The fused step's attention phase gives each (sequence,
+    quarter of D) unit SMs // (4 * B) CTAs; measured on B200 it wins with
+    at least four per unit (4 sequences: 58 vs 61 us per 1M-context step)
+    and loses with two (16 sequences: 76 vs 63 us per 64K-context step)."""
+    sms = torch.cuda.get_device_properties(device or torch.cuda.current_device()).multi_processor_count
+    return 16 * B <= sms
+
+
 def _ws(nbytes: int, device) -> torch.Tensor | None:
     return torch.empty(nbytes, dtype=torch.uint8, device=device) if nbytes else None
 
@@ -75,14 +85,14 @@ class DecodeState:
     window ring.  Capacity is fixed at construction (``entry_cap`` entries).
 
     ``dense=True`` makes it an HCA cache (no indexer, dense attention).
-    ``fused=True`` (the default) runs each CSA step as one csa_decode_step
-    launch where the shape allows it; ``fused=False`` always uses the
-    separate calls.
+    ``fused=True`` runs each CSA step as one csa_decode_step launch where
+    the shape allows it; ``fused=False`` always uses the separate calls;
+    ``fused=None`` (the default) picks by :func:`prefer_fused_step`.
     """
 
     def __init__(self, B: int, D: int, H: int, m: int, W: int, entry_cap: int, *, K: int = 512,
                  HI: int = 4, dI: int = 64, win_cap: int | None = None, dense: bool = False,
-                 softmax_scale: float = 1.0, device="cuda", fused: bool = True):
+                 softmax_scale: float = 1.0, device="cuda", fused: bool | None = None):
         self.B, self.D, self.H, self.m, self.W, self.K = B, D, H, m, W, K
         self.HI, self.dI, self.dense = HI, dI, dense
         self.win_cap = W if win_cap is None else win_cap
@@ -105,6 +115,8 @@ class DecodeState:
         self._ws_attend = None
         self._ws_step = None
         self._side = None
+        if fused is None:
+            fused = prefer_fused_step(B, self.device)
         self.fused = fused and not dense
 
     @property
