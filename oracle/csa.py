@@ -44,6 +44,11 @@ Readings where the pages are silent (this library's contract)
   with E2M1 qI, kI and w a multiple of 1/16 in [0, 1].  Every product of two
   E2M1 values is a multiple of 1/4, so 64 * score is an integer; the oracle
   computes that integer exactly.
+* Block-scaled indexer (MXFP4 queries and keys, each 32-element block with
+  its own E8M0 power-of-two scale): the same score, no longer an exact
+  integer; a fixed-precision evaluation differs from it by at most a small
+  multiple of the rounding unit times mag = sum_h w_h sum_j |q_hj k_j|, so
+  entries whose scores lie that close to the k-th may swap places.
 * Top-k: the K highest scores among visible entries, ties to the lower
   index; fewer than K visible -> all of them; rows are in rank order
   (score descending, index ascending) and padded with -1.
@@ -178,6 +183,63 @@ def indexer_scores64(qI_packed, w, kI_packed) -> np.ndarray:
         dots = dots.astype(np.int64).reshape(Tq, H, N)
         out[b] = (w16[b][:, :, None] * np.maximum(dots, 0)).sum(axis=1)
     return out
+
+
+# --------------------------------------------------------------------------
+# (2b) Lightning Indexer on block-scaled FP4 (MXFP4) queries and keys
+# --------------------------------------------------------------------------
+
+
+def mx_values(packed, scale_codes) -> np.ndarray:
+    """MXFP4 rows to float64: element j of a row is its E2M1 value times
+    2**(E8M0 code of block j // 32 - 127).
+
+    packed: u8 [..., d/2]; scale_codes: u8 [..., d/32].  Exact in float64.
+    Pages: studioglobal.ai "FP4/FP8混合精度" (MXFP4, two values per byte);
+    jiwasawa "限界を押し広げるインフラストラクチャの最適化" (FP4 on the
+    indexer's QK path).
+    """
+    v = e2m1_decode(e2m1_unpack(packed))
+    sc = np.asarray(scale_codes).astype(np.int64)
+    if (sc == 0xFF).any():
+        raise ValueError("E8M0 code 0xFF (NaN) is not a scale")
+    f = np.exp2((sc - 127).astype(np.float64))
+    return v * np.repeat(f, 32, axis=-1)
+
+
+def indexer_scores_mx(qI_packed, qI_scales, w, kI_packed, kI_scales):
+    """Indexer scores on MXFP4 queries and keys, and the magnitude their
+    rounding error scales with.
+
+    qI_packed u8 [B, Tq, H_I, d_I/2], qI_scales u8 [B, Tq, H_I, d_I/32];
+    w f32 [B, Tq, H_I] (non-negative); kI_packed u8 [B, N, d_I/2],
+    kI_scales u8 [B, N, d_I/32].
+    Returns float64 [B, Tq, N] pairs (score, mag):
+        score = sum_h w_h * max(0, sum_j q_hj k_j)
+        mag   = sum_h w_h * sum_j |q_hj k_j|
+    Within one 32-element block every product is a multiple of the same
+    power of two and the block's sum is exact in float64; only the sum over
+    blocks and heads rounds, at float64 precision.  Pages: jiwasawa
+    "Compressed Sparse Attention (CSA)" (the indexer's score),
+    "限界を押し広げるインフラストラクチャの最適化" (FP4 QK path);
+    studioglobal.ai "FP4/FP8混合精度" (MXFP4).
+    """
+    q = mx_values(qI_packed, qI_scales)          # [B, Tq, H, d]
+    k = mx_values(kI_packed, kI_scales)          # [B, N, d]
+    w = np.asarray(w, dtype=np.float32).astype(np.float64)
+    if (w < 0).any() or not np.isfinite(w).all():
+        raise ValueError("indexer weights must be finite and non-negative")
+    B, Tq, H, d = q.shape
+    N = k.shape[1]
+    score = np.zeros((B, Tq, N))
+    mag = np.zeros((B, Tq, N))
+    for b in range(B):
+        qq = q[b].reshape(Tq * H, d)
+        dots = (qq @ k[b].T).reshape(Tq, H, N)
+        absd = (np.abs(qq) @ np.abs(k[b]).T).reshape(Tq, H, N)
+        score[b] = (w[b][:, :, None] * np.maximum(dots, 0.0)).sum(axis=1)
+        mag[b] = (w[b][:, :, None] * absd).sum(axis=1)
+    return score, mag
 
 
 # --------------------------------------------------------------------------

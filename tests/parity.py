@@ -16,6 +16,21 @@ contract):
   1e-2 * max_d |ref|.
 * log-sum-exp: |gpu - ref| <= 1e-4 (logits are exact products of bf16 and
   E4M3 values accumulated in fp32; exp2/log2 add a few ulp).
+* block-scaled (MXFP4) indexer scores: |gpu - ref| <= MX_RTOL * mag with
+  mag = sum_h w_h sum_j |q_hj k_j| (the oracle's second output).  The
+  kernel's arithmetic: within a 32-element block the products share one
+  power of two and their sum has at most 11 significant bits, exact in any
+  fp32 accumulator; the tensor core then adds the two scaled block sums
+  (its internal accumulation precision is not documented, so allow 2^-12
+  relative to the magnitude rather than fp32's 2^-24), and the epilogue's
+  relu, weight and sum over heads round three or four more times in fp32.
+  MX_RTOL = 2^-12 covers all of it.
+* block-scaled top-k (tie-tolerant): the k listed entries are distinct and
+  visible, padded with -1, their reported scores within the score bound and
+  non-increasing; and no left-out entry can beat a listed one: for every
+  listed e and unlisted f, ref(e) + err(e) >= ref(f) - err(f).  Entries
+  whose scores lie within the bounds of the k-th may therefore swap, and
+  nothing else may.
 """
 from __future__ import annotations
 
@@ -27,6 +42,7 @@ from oracle.formats import e4m3_decode
 POOL_RTOL = 1e-5
 OUT_RTOL = 1e-2
 LSE_ATOL = 1e-4
+MX_RTOL = 2.0 ** -12
 
 
 def pooled_and_scale(x, z, m):
@@ -94,3 +110,40 @@ def check_attention(gpu_out_bf16, gpu_lse, ref_out, ref_lse):
         lerr = np.abs(gl - ref_lse)
         assert lerr.max() <= LSE_ATOL, f"lse mismatch: max err {lerr.max():.3g}"
     return float((err / scale).max())
+
+
+def check_topk_tolerant(gpu_idx, gpu_score, ref_score, mag, n_vis, K, rtol=MX_RTOL):
+    """Tie-tolerant check of one block of rows.
+
+    gpu_idx int [R, K], gpu_score [R, K] (or None), ref_score / mag float64
+    [R, N] from the oracle, n_vis [R].  Raises AssertionError naming the
+    first violated rule; returns the number of rows whose list differs from
+    the oracle's exact rank order (near-ties that swapped).
+    """
+    gpu_idx = np.asarray(gpu_idx)
+    swapped = 0
+    for r in range(gpu_idx.shape[0]):
+        nv = int(n_vis[r])
+        k = min(K, nv)
+        g = gpu_idx[r]
+        assert (g[k:] == -1).all(), f"row {r}: padding past {k} entries"
+        sel = g[:k].astype(np.int64)
+        assert ((sel >= 0) & (sel < nv)).all(), f"row {r}: an index outside the {nv} visible entries"
+        assert np.unique(sel).size == k, f"row {r}: repeated index"
+        ref = np.asarray(ref_score[r, :nv], dtype=np.float64)
+        err = rtol * np.asarray(mag[r, :nv], dtype=np.float64)
+        if gpu_score is not None:
+            gs = np.asarray(gpu_score[r], dtype=np.float64)
+            assert (np.abs(gs[:k] - ref[sel]) <= err[sel] + 1e-30).all(), f"row {r}: a score outside its bound"
+            assert (np.diff(gs[:k]) <= 0).all(), f"row {r}: scores not in descending order"
+            assert (gs[k:] == 0).all(), f"row {r}: padding score not 0"
+        if k < nv:
+            rest = np.ones(nv, dtype=bool)
+            rest[sel] = False
+            lo_sel = (ref[sel] + err[sel]).min()
+            hi_rest = (ref[rest] - err[rest]).max()
+            assert lo_sel >= hi_rest, (f"row {r}: a left-out entry beats a listed one "
+                                       f"({hi_rest:.9g} > {lo_sel:.9g})")
+        exact = np.lexsort((np.arange(nv), -ref))[:k]
+        swapped += int(not np.array_equal(exact, sel))
+    return swapped
