@@ -30,6 +30,8 @@ SYMBOLS = (
     "csa_index_topk_workspace",
     "csa_index_topk",
     "csa_index_topk_noalloc",
+    "csa_index_topk_mx_workspace",
+    "csa_index_topk_mx",
     "csa_attend_workspace",
     "csa_attend",
     "hca_attend_workspace",
@@ -93,6 +95,10 @@ def lib() -> ctypes.CDLL:
     L.csa_index_topk.restype = ctypes.c_int
     L.csa_index_topk_noalloc.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P]
     L.csa_index_topk_noalloc.restype = ctypes.c_int
+    L.csa_index_topk_mx_workspace.argtypes = [ctypes.POINTER(Dims)]
+    L.csa_index_topk_mx_workspace.restype = _SZ
+    L.csa_index_topk_mx.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
+    L.csa_index_topk_mx.restype = ctypes.c_int
     for name in ("csa_attend_workspace", "hca_attend_workspace"):
         getattr(L, name).argtypes = [ctypes.POINTER(Dims)]
         getattr(L, name).restype = _SZ
@@ -195,6 +201,10 @@ def index_topk_workspace(dims: Dims) -> int:
     return int(lib().csa_index_topk_workspace(ctypes.byref(dims)))
 
 
+def index_topk_mx_workspace(dims: Dims) -> int:
+    return int(lib().csa_index_topk_mx_workspace(ctypes.byref(dims)))
+
+
 def attend_workspace(dims: Dims, dense: bool = False) -> int:
     fn = lib().hca_attend_workspace if dense else lib().csa_attend_workspace
     return int(fn(ctypes.byref(dims)))
@@ -229,6 +239,20 @@ def index_topk_noalloc(qI, w, kI, q_pos, dims: Dims, idx_out, score_out=None, st
                                         _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
                                         _ptr(idx_out, torch.int32, "idx_out", dev),
                                         _ptr(score_out, torch.float32, "score_out", dev), _stream(stream)))
+
+
+def index_topk_mx(qI, qI_scales, w, kI, kI_scales, q_pos, dims: Dims, idx_out, score_out=None, workspace=None,
+                  stream=None):
+    """csa_index_topk_mx: indexer + top-k on block-scaled FP4 (MXFP4) queries
+    and keys; see include/csa.h."""
+    dev = qI.device
+    wp, wn = _ws(workspace, index_topk_mx_workspace(dims), dev)
+    _check(lib().csa_index_topk_mx(_ptr(qI, torch.uint8, "qI"), _ptr(qI_scales, torch.uint8, "qI_scales", dev),
+                                   _ptr(w, torch.float32, "w", dev), _ptr(kI, torch.uint8, "kI", dev),
+                                   _ptr(kI_scales, torch.uint8, "kI_scales", dev),
+                                   _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims),
+                                   _ptr(idx_out, torch.int32, "idx_out", dev),
+                                   _ptr(score_out, torch.float32, "score_out", dev), wp, wn, _stream(stream)))
 
 
 def attend(q, codes, scales, idx, win_codes, win_scales, q_pos, dims: Dims, out, lse=None,

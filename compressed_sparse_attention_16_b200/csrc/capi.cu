@@ -276,6 +276,35 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t csa_index_topk_mx_workspace(const csa_dims *d) {
+  if (!d || d->B < 0 || d->Tq < 0 || d->n_entries < 0) return 0;
+  return index_mx_workspace(d);
+}
+
+int csa_index_topk_mx(const uint8_t *qI, const uint8_t *qI_scales, const float *w, const uint8_t *kI,
+                      const uint8_t *kI_scales, const int32_t *q_pos, const csa_dims *d, int32_t *idx_out,
+                      float *score_out, void *workspace, size_t workspace_bytes, csa_stream_t stream) {
+  clear_error();
+  if (int rc = check_index_dims("csa_index_topk_mx", d)) return rc;
+  if ((int64_t)d->B * d->Tq == 0) return CSA_OK;
+  if (!qI || !qI_scales || !w || !kI || !kI_scales || !q_pos || !idx_out)
+    return fail(CSA_ERR_INVALID, "csa_index_topk_mx: NULL buffer");
+  if (!aligned16(kI) || !aligned16(qI) || ((uintptr_t)w & 3) || ((uintptr_t)q_pos & 3) ||
+      ((uintptr_t)idx_out & 3) || ((uintptr_t)score_out & 3))
+    return fail(CSA_ERR_INVALID, "csa_index_topk_mx: misaligned buffer");
+  int splits, slice;
+  if (!index_mx_plan(d, &splits, &slice))
+    return fail(CSA_ERR_UNSUPPORTED, "csa_index_topk_mx: dI=%d HI=%d K=%d n_entries=%d (supported: dI 64, HI 1..8, "
+                "at most 20,480 / K slices of 4,096 entries)", d->dI, d->HI, d->K, d->n_entries);
+  const size_t need = index_mx_workspace(d);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(CSA_ERR_WORKSPACE, "csa_index_topk_mx: workspace needs %zu bytes (got %zu)", need,
+                workspace_bytes);
+  if (int rc = need_status()) return rc;
+  return launch_index_mx(qI, qI_scales, w, kI, kI_scales, q_pos, d, idx_out, score_out, workspace,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t csa_attend_workspace(const csa_dims *d) { return d ? attend_workspace(d, false) : 0; }
 size_t hca_attend_workspace(const csa_dims *d) { return d ? attend_workspace(d, true) : 0; }
 
@@ -366,7 +395,7 @@ int csa_sync_status(csa_stream_t stream) {
   if (v & STATUS_TIMEOUT) return fail(CSA_ERR_TIMEOUT, "a device-side wait timed out (status 0x%x)", v);
   if (v & (STATUS_BAD_WEIGHT | STATUS_BAD_INDEX | STATUS_BAD_POSITION))
     return fail(CSA_ERR_INVALID, "invalid device data: %s%s%s (status 0x%x)",
-                (v & STATUS_BAD_WEIGHT) ? "indexer weight off the 1/16 grid; " : "",
+                (v & STATUS_BAD_WEIGHT) ? "indexer weight off its grid or a NaN block scale; " : "",
                 (v & STATUS_BAD_INDEX) ? "attention index out of range; " : "",
                 (v & STATUS_BAD_POSITION) ? "negative query position" : "", v);
   return CSA_OK;

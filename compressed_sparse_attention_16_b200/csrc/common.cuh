@@ -21,13 +21,25 @@ void count_launches(unsigned n);   // bookkeeping for csa_launch_count()
 void clear_error();
 // Host checks of a csa_index_topk shape (CSA_OK or the error, message set).
 int check_index_dims(const char *fn, const csa_dims *d);
+// The K best of each row's splits x K candidate keys in rank order (scores
+// as 64 * score integers, or fp32 bits when float_scores).
+int launch_topk_merge(const uint64_t *cand, int splits, const csa_dims *d, const int32_t *q_pos, int32_t *idx_out,
+                      float *score_out, bool float_scores, cudaStream_t stream);
+// The block-scaled (MXFP4) indexer: plan, workspace bytes (0 when the shape
+// is outside the plan), launch.
+bool index_mx_plan(const csa_dims *d, int *splits, int *slice);
+size_t index_mx_workspace(const csa_dims *d);
+int launch_index_mx(const uint8_t *qI, const uint8_t *qs, const float *w, const uint8_t *kI, const uint8_t *ks,
+                    const int32_t *q_pos, const csa_dims *d, int32_t *idx_out, float *score_out, void *workspace,
+                    cudaStream_t stream);
 
 // ---------------------------------------------------------------------------
 // device status word (set by kernels, read + cleared by csa_sync_status)
 // ---------------------------------------------------------------------------
 enum : unsigned {
   STATUS_TIMEOUT = 1u,      // a bounded wait gave up
-  STATUS_BAD_WEIGHT = 2u,   // indexer weight not a multiple of 1/16 in [0, 1]
+  STATUS_BAD_WEIGHT = 2u,   // indexer weight off its grid (1/16 steps in [0, 1]; block-scaled: negative or
+                            // not finite, or an E8M0 scale of 0xFF)
   STATUS_BAD_INDEX = 4u,    // attention index outside [0, n_entries) other than -1
   STATUS_BAD_POSITION = 8u, // negative query position (treated as position 0 / no entries)
 };

@@ -23,6 +23,7 @@
 // bitonic network.
 #include "common.cuh"
 #include "tc.cuh"
+#include "select.cuh"
 
 namespace csa {
 namespace {
@@ -394,101 +395,10 @@ constexpr int kSliceMax = 8192;
 constexpr int kMergeThreads = 1024;
 constexpr int kMergeCap = 20480;     // candidate keys per row held by the merge CTA (160 KiB)
 
-// Bin (0..4095) where the count of keys in this-or-higher bins first reaches
-// `need`, and the count strictly above it.  NT threads, 4096/NT bins each.
-template <int NT>
-__device__ void find_bin(const uint32_t *hist, uint32_t need, uint32_t *warp_tot, int *out_bin,
-                         uint32_t *out_above) {
-  constexpr int BPT = kBins / NT;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hi_bin = kBins - 1 - BPT * tid;
-  uint32_t c[BPT], local = 0;
-  if (((uintptr_t)hist & 15u) == 0) {
-    // this thread's BPT bins are contiguous and 16-byte aligned: vector loads
-    // (scalar loads at a stride of BPT words would conflict on the banks)
-    const uint4 *h4 = reinterpret_cast<const uint4 *>(hist + hi_bin - (BPT - 1));
-#pragma unroll
-    for (int k4 = 0; k4 < BPT / 4; ++k4) {
-      const uint4 v = h4[k4];
-      c[BPT - 1 - 4 * k4] = v.x;
-      c[BPT - 2 - 4 * k4] = v.y;
-      c[BPT - 3 - 4 * k4] = v.z;
-      c[BPT - 4 - 4 * k4] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < BPT; ++k) c[k] = hist[hi_bin - k];
-  }
-#pragma unroll
-  for (int k = 0; k < BPT; ++k) local += c[k];
-  uint32_t v = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += x;
-  }
-  if (lane == 31) warp_tot[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t wv = lane < NT / 32 ? warp_tot[lane] : 0u;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, wv, o);
-      if (lane >= o) wv += x;
-    }
-    if (lane < NT / 32) warp_tot[lane] = wv;
-  }
-  __syncthreads();
-  const uint32_t incl = v + (warp > 0 ? warp_tot[warp - 1] : 0u);
-  const uint32_t excl = incl - local;
-  if (excl < need && incl >= need) {
-    uint32_t run = excl;
-#pragma unroll
-    for (int k = 0; k < BPT; ++k) {
-      if (run + c[k] >= need) { *out_bin = hi_bin - k; *out_above = run; break; }
-      run += c[k];
-    }
-  }
-  __syncthreads();
-}
-
-struct SelShared {
-  uint32_t warp_tot[32];
-  int bin;
-  uint32_t above;
-  uint32_t count;
-};
-
-// Threshold T such that exactly K of the n keys are >= T (keys distinct, K <= n):
-// radix select over the key bits, 12 bits per pass, stopping as soon as the
-// threshold bin is taken whole.
-template <int NT>
-__device__ uint64_t kth_largest_key(const uint64_t *keys, int n, int K, uint32_t *hist, SelShared *sh) {
-  uint64_t prefix = 0, pmask = 0;
-  uint32_t need = (uint32_t)K;
-  const int shifts[5] = {44, 32, 20, 8, 0};
-  const uint32_t dmask[5] = {0xFFFu, 0xFFFu, 0xFFFu, 0xFFFu, 0xFFu};
-  for (int dgt = 0; dgt < 5; ++dgt) {
-    const int sft = shifts[dgt];
-    const uint32_t dm = dmask[dgt];
-    for (int i = threadIdx.x; i < kBins; i += NT) hist[i] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < n; j += NT) {
-      const uint64_t k = keys[j];
-      if ((k & pmask) == prefix) atomicAdd(&hist[(uint32_t)(k >> sft) & dm], 1u);
-    }
-    __syncthreads();
-    find_bin<NT>(hist, need, sh->warp_tot, &sh->bin, &sh->above);
-    const uint32_t bin = (uint32_t)sh->bin;
-    need -= sh->above;
-    prefix |= (uint64_t)bin << sft;
-    pmask |= (uint64_t)dm << sft;
-    const uint32_t in_bin = hist[bin];
-    __syncthreads();
-    if (in_bin == need) break;       // the whole bin is taken: keys >= prefix
-  }
-  return prefix;
-}
+using sel::find_bin;
+using sel::kth_largest_key;
+using sel::SelShared;
+static_assert(kBins == sel::kSelBins, "selection bins");
 
 template <int HI, int DI>
 __global__ void __launch_bounds__(kPartThreads)
@@ -546,6 +456,9 @@ index_partial_kernel(const uint8_t *__restrict__ qI, const float *__restrict__ w
   }
 }
 
+// WIDE: the keys carry fp32 score bits (the block-scaled indexer) rather
+// than 64 * score as an integer below 2^24.
+template <bool WIDE>
 __global__ void __launch_bounds__(kMergeThreads)
 topk_merge_kernel(const uint64_t *__restrict__ cand, int splits, int K, const int32_t *__restrict__ q_pos,
                   int m, int n_entries, int32_t *__restrict__ idx_out, float *__restrict__ score_out) {
@@ -564,7 +477,7 @@ topk_merge_kernel(const uint64_t *__restrict__ cand, int splits, int K, const in
   __syncthreads();
   const int cnt = min(K, nvis);
   // real candidates are non-zero keys; padding keys are 0 and rank last
-  const uint64_t T = (nvis > K) ? kth_largest_key<kMergeThreads>(keys, n, K, hist, sh) : 1ull;
+  const uint64_t T = (nvis > K) ? kth_largest_key<kMergeThreads, WIDE>(keys, n, K, hist, sh) : 1ull;
   for (int j = tid; j < n; j += kMergeThreads) {
     const uint64_t k = keys[j];
     if (k >= T) best[atomicAdd(&sh->count, 1u)] = k;
@@ -581,7 +494,7 @@ topk_merge_kernel(const uint64_t *__restrict__ cand, int splits, int K, const in
     if (j < cnt) {
       const uint64_t k = best[j];
       id = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFu));
-      sc = (float)(uint32_t)(k >> 32) * (1.f / 64.f);
+      sc = WIDE ? __uint_as_float((uint32_t)(k >> 32)) : (float)(uint32_t)(k >> 32) * (1.f / 64.f);
     }
     idx_out[(int64_t)row * K + j] = id;
     if (score_out) score_out[(int64_t)row * K + j] = sc;
@@ -1803,6 +1716,23 @@ int launch_prefill_tc(const uint8_t *qI, const float *w, const uint8_t *kI, cons
 
 }  // namespace
 
+// The K best of each row's splits x K candidate keys, in rank order.
+int launch_topk_merge(const uint64_t *cand, int splits, const csa_dims *d, const int32_t *q_pos, int32_t *idx_out,
+                      float *score_out, bool float_scores, cudaStream_t stream) {
+  const int64_t rows = (int64_t)d->B * d->Tq;
+  const size_t smem = (kMergeCap + kMaxK) * 8 + kBins * 4 + sizeof(SelShared);
+  const void *fn = float_scores ? (const void *)topk_merge_kernel<true> : (const void *)topk_merge_kernel<false>;
+  if (int rc = set_smem_once(fn, (int)smem, "topk_merge_kernel")) return rc;
+  if (float_scores)
+    topk_merge_kernel<true><<<rows, kMergeThreads, smem, stream>>>(cand, splits, d->K, q_pos, d->m, d->n_entries,
+                                                                   idx_out, score_out);
+  else
+    topk_merge_kernel<false><<<rows, kMergeThreads, smem, stream>>>(cand, splits, d->K, q_pos, d->m, d->n_entries,
+                                                                    idx_out, score_out);
+  count_launches(1);
+  return check_launch("topk_merge_kernel");
+}
+
 bool prefill2_plan(const csa_dims *d);
 size_t prefill2_workspace(const csa_dims *d);
 int launch_prefill2(const uint8_t *qI, const float *w, const uint8_t *kI, const int32_t *q_pos, const csa_dims *d,
@@ -1852,12 +1782,7 @@ int launch_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, cons
     }
 #undef CSA_PARTIAL
     if (int rc = check_launch("index_partial_kernel")) return rc;
-    const size_t smem = (kMergeCap + kMaxK) * 8 + kBins * 4 + sizeof(SelShared);
-    if (int rc = set_smem_once((const void *)topk_merge_kernel, (int)smem, "topk_merge_kernel")) return rc;
-    topk_merge_kernel<<<rows, kMergeThreads, smem, stream>>>(cand, splits, d->K, q_pos, d->m, d->n_entries,
-                                                             idx_out, score_out);
-    count_launches(1);
-    return check_launch("topk_merge_kernel");
+    return launch_topk_merge(cand, splits, d, q_pos, idx_out, score_out, false, stream);
   }
   const int64_t ld = ((int64_t)d->n_entries + 3) & ~3LL;
   uint32_t *scores = static_cast<uint32_t *>(workspace);

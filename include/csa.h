@@ -149,6 +149,44 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
                    size_t workspace_bytes, csa_stream_t stream);
 
 /*
+ * csa_index_topk_mx -- the indexer and top-k on block-scaled FP4 (MXFP4)
+ * queries and keys.
+ * (jiwasawa "限界を押し広げるインフラストラクチャの最適化": FP4 on the
+ *  indexer's QK path; studioglobal.ai "FP4/FP8混合精度": MXFP4, two values per
+ *  byte; jiwasawa "Compressed Sparse Attention (CSA)": indexer + top-k.)
+ *
+ * Element j of a query head or key row is its E2M1 code times
+ * 2^(s - 127), s the row's UE8M0 scale code for block j / 32 (the output of
+ * csa_quantize_mxfp4).  For query row (b, i) at position t and visible entry
+ * s (as csa_index_topk):
+ *     score = sum_h w[b,i,h] * max(0, sum_j q[b,i,h,j] * k[b,s,j])
+ * evaluated on the tensor cores with the block scales applied in the MMA and
+ * fp32 accumulation: not exact.  The listed entries are the k best by the
+ * computed fp32 score (ties to the lower index), in rank order, -1 padding;
+ * entries whose exact scores lie within the evaluation's rounding of the
+ * k-th may be listed in place of one another.
+ *
+ *   qI         u8 [B, Tq, HI, 32]  packed E2M1 (dI = 64), 16-byte aligned
+ *   qI_scales  u8 [B, Tq, HI, 2]   UE8M0 codes (0xFF, NaN, is reported)
+ *   w          fp32 [B, Tq, HI]    finite, >= 0 (else reported and taken as 0)
+ *   kI         u8 [B, entry_cap, 32], 16-byte aligned
+ *   kI_scales  u8 [B, entry_cap, 2]
+ *   q_pos, idx_out as csa_index_topk; score_out fp32 [B, Tq, K] (the
+ *   computed scores, 0 for padding) or NULL
+ *   workspace  at least csa_index_topk_mx_workspace(d) bytes
+ * Supported: dI = 64, HI 1..8, K 1..2048, and at most 20,480 / K slices of
+ * 4,096 entries per row (n_entries <= 163,840 at K = 512); otherwise
+ * CSA_ERR_UNSUPPORTED before any launch.  Negative weights, non-finite
+ * weights and 0xFF scales set a status bit (csa_sync_status ->
+ * CSA_ERR_INVALID).  The workspace query returns 0 for unsupported shapes.
+ */
+size_t csa_index_topk_mx_workspace(const csa_dims *d);
+int csa_index_topk_mx(const uint8_t *qI, const uint8_t *qI_scales, const float *w, const uint8_t *kI,
+                      const uint8_t *kI_scales, const int32_t *q_pos, const csa_dims *d,
+                      int32_t *idx_out, float *score_out, void *workspace, size_t workspace_bytes,
+                      csa_stream_t stream);
+
+/*
  * csa_index_topk_noalloc -- csa_index_topk without a caller-provided workspace.
  * (The pages have no counterpart: this is a deployment convenience.)
  *

@@ -163,3 +163,34 @@ def indexer_inputs(B: int, Tq: int, Ncap: int, HI: int, dI: int, seed: int, devi
         w=indexer_weights(B, Tq, HI, seed, device),
         kI=e2m1_packed((B, Ncap), dI, seed, "kI", device),
     )
+
+
+@dataclasses.dataclass
+class IndexerInputsMX:
+    qI: torch.Tensor   # u8 [B, Tq, HI, dI/2]  E2M1 codes
+    qs: torch.Tensor   # u8 [B, Tq, HI, dI/32] UE8M0 block scales
+    w: torch.Tensor    # f32 [B, Tq, HI]        non-negative
+    kI: torch.Tensor   # u8 [B, Ncap, dI/2]
+    ks: torch.Tensor   # u8 [B, Ncap, dI/32]
+
+
+def ue8m0_codes(shape, seed: int, tag: str, device="cpu", spread: int = 8) -> torch.Tensor:
+    """Block scale codes 127 + u, u uniform in [-spread, spread] (scales
+    2^-spread .. 2^spread around 1)."""
+    g = _gen(seed, tag + ":scales", device)
+    u = torch.randint(-spread, spread + 1, shape, generator=g, device=device, dtype=torch.int32)
+    return (127 + u).to(torch.uint8)
+
+
+def indexer_inputs_mx(B: int, Tq: int, Ncap: int, HI: int, dI: int, seed: int, device="cpu",
+                      spread: int = 8) -> IndexerInputsMX:
+    """MXFP4 indexer inputs: E2M1 codes as `indexer_inputs`, one UE8M0 scale
+    per 32 elements drawn by `ue8m0_codes`, weights uniform in [0, 1)."""
+    g = _gen(seed, "wmx", device)
+    return IndexerInputsMX(
+        qI=e2m1_packed((B, Tq, HI), dI, seed, "qI", device),
+        qs=ue8m0_codes((B, Tq, HI, dI // 32), seed, "qI", device, spread),
+        w=torch.rand((B, Tq, HI), generator=g, device=device),
+        kI=e2m1_packed((B, Ncap), dI, seed, "kI", device),
+        ks=ue8m0_codes((B, Ncap, dI // 32), seed, "kI", device, spread),
+    )

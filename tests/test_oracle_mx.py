@@ -148,7 +148,7 @@ def test_tolerant_check_on_oracle_output_with_bounded_perturbation():
     exact = np.stack([_exact_topk(ref[r], nv[r], K) for r in range(Tq)])
     ex_sc = np.where(exact >= 0, np.take_along_axis(ref, np.maximum(exact, 0), axis=1), 0.0)
     assert check_topk_tolerant(exact, ex_sc, ref, mag[0], nv, K) == 0
-    noisy = ref + (rng.random(ref.shape) * 2 - 1) * 2 ** -13 * mag[0]
+    noisy = ref + (rng.random(ref.shape) * 2 - 1) * 2 ** -21 * mag[0]
     pert = np.stack([_exact_topk(noisy[r], nv[r], K) for r in range(Tq)])
     pert_sc = np.where(pert >= 0, np.take_along_axis(noisy, np.maximum(pert, 0), axis=1), 0.0)
     check_topk_tolerant(pert, pert_sc, ref, mag[0], nv, K)
