@@ -15,7 +15,9 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libcsa.so")
+# the library to load: libcsa.so, or another build (the CSA_CHECK build
+# libcsa_check.so) named by the CSA_LIBRARY environment variable
+LIB_PATH = os.environ.get("CSA_LIBRARY") or os.path.join(_HERE, "libcsa.so")
 
 CSA_OK = 0
 CSA_ERR_INVALID = -1
@@ -23,6 +25,7 @@ CSA_ERR_UNSUPPORTED = -2
 CSA_ERR_CUDA = -3
 CSA_ERR_TIMEOUT = -4
 CSA_ERR_WORKSPACE = -5
+CSA_ERR_CHECK = -6
 
 # every symbol declared in include/csa.h
 SYMBOLS = (
@@ -32,6 +35,8 @@ SYMBOLS = (
     "csa_index_topk_noalloc",
     "csa_index_topk_mx_workspace",
     "csa_index_topk_mx",
+    "csa_check_topk",
+    "csa_check_build",
     "csa_attend_workspace",
     "csa_attend",
     "hca_attend_workspace",
@@ -99,6 +104,10 @@ def lib() -> ctypes.CDLL:
     L.csa_index_topk_mx_workspace.restype = _SZ
     L.csa_index_topk_mx.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
     L.csa_index_topk_mx.restype = ctypes.c_int
+    L.csa_check_topk.argtypes = [_P, _P, _P, ctypes.POINTER(Dims), _P]
+    L.csa_check_topk.restype = ctypes.c_int
+    L.csa_check_build.argtypes = []
+    L.csa_check_build.restype = ctypes.c_int
     for name in ("csa_attend_workspace", "hca_attend_workspace"):
         getattr(L, name).argtypes = [ctypes.POINTER(Dims)]
         getattr(L, name).restype = _SZ
@@ -203,6 +212,19 @@ def index_topk_workspace(dims: Dims) -> int:
 
 def index_topk_mx_workspace(dims: Dims) -> int:
     return int(lib().csa_index_topk_mx_workspace(ctypes.byref(dims)))
+
+
+def check_topk(idx, score, q_pos, dims: Dims, stream=None) -> None:
+    """csa_check_topk: device-side check of top-k lists; a violation is
+    reported by the next sync_status() (CSA_ERR_CHECK)."""
+    dev = idx.device
+    _check(lib().csa_check_topk(_ptr(idx, torch.int32, "idx"), _ptr(score, torch.float32, "score", dev),
+                                _ptr(q_pos, torch.int32, "q_pos", dev), ctypes.byref(dims), _stream(stream)))
+
+
+def is_check_build() -> bool:
+    """True when the loaded library is the CSA_CHECK build."""
+    return bool(lib().csa_check_build())
 
 
 def attend_workspace(dims: Dims, dense: bool = False) -> int:

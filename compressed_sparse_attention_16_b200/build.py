@@ -1,8 +1,10 @@
 """Build libcsa.so in-tree from csrc/*.cu with nvcc for sm_100a.
 
-Usage: python -m compressed_sparse_attention_16_b200.build [--force] [-v]
+Usage: python -m compressed_sparse_attention_16_b200.build [--force] [-v] [--check]
 The shared library links the CUDA runtime statically, so it needs only the
-NVIDIA driver at run time.
+NVIDIA driver at run time.  --check also builds libcsa_check.so, the
+CSA_CHECK build (the C API file compiled with -DCSA_CHECK, every other
+object shared), which checks every top-k list it writes on the device.
 """
 from __future__ import annotations
 
@@ -77,6 +79,32 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     return LIB
 
 
+CHECK_LIB = os.path.join(HERE, "libcsa_check.so")
+
+
+def build_check(force: bool = False, verbose: bool = False) -> str:
+    """The CSA_CHECK build: capi.cu with -DCSA_CHECK, linked with the default
+    build's other objects (built first if needed)."""
+    build(force=force, verbose=verbose)
+    nvcc = _nvcc()
+    capi = os.path.join(CSRC, "capi.cu")
+    obj = os.path.join(OBJDIR, "capi_check.o")
+    objs = [os.path.join(OBJDIR, os.path.basename(s)[:-3] + ".o") for s in sources() if s != capi]
+    if force or _stale(obj, [capi] + _deps()):
+        cmd = [nvcc] + ARCH + CFLAGS + ["-DCSA_CHECK", "-c", capi, "-o", obj]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
+    if force or _stale(CHECK_LIB, objs + [obj]):
+        cmd = [nvcc] + ARCH + ["-shared", "-cudart", "static", "-o", CHECK_LIB] + objs + [obj]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError("nvcc link failed:\n" + r.stdout + r.stderr)
+    return CHECK_LIB
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose="-v" in sys.argv)
     print(LIB)
+    if "--check" in sys.argv:
+        print(build_check(verbose="-v" in sys.argv))

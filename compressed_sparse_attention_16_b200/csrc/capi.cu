@@ -209,9 +209,38 @@ int check_index_dims(const char *fn, const csa_dims *d) {
     return fail(CSA_ERR_UNSUPPORTED, "%s: HI=%d dI=%d", fn, d->HI, d->dI);
   return CSA_OK;
 }
+// The CSA_CHECK build checks every top-k list the library writes; the
+// default build does not.
+static int debug_check_topk(const int32_t *idx, const float *score, const int32_t *q_pos, const csa_dims *d,
+                            cudaStream_t stream) {
+#ifdef CSA_CHECK
+  return launch_check_topk(idx, score, q_pos, d, stream);
+#else
+  (void)idx; (void)score; (void)q_pos; (void)d; (void)stream;
+  return CSA_OK;
+#endif
+}
 }  // namespace csa
 
 extern "C" {
+
+int csa_check_build(void) {
+#ifdef CSA_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int csa_check_topk(const int32_t *idx, const float *score, const int32_t *q_pos, const csa_dims *d,
+                   csa_stream_t stream) {
+  clear_error();
+  if (!d || !idx || !q_pos || d->B < 0 || d->Tq < 0 || d->m < 1 || d->K < 1 || d->n_entries < 0)
+    return fail(CSA_ERR_INVALID, "csa_check_topk: bad arguments");
+  if (((uintptr_t)idx & 3) || ((uintptr_t)score & 3) || ((uintptr_t)q_pos & 3))
+    return fail(CSA_ERR_INVALID, "csa_check_topk: misaligned buffer");
+  return launch_check_topk(idx, score, q_pos, d, reinterpret_cast<cudaStream_t>(stream));
+}
 
 int csa_version(void) { return 100; }
 
@@ -272,8 +301,9 @@ int csa_index_topk(const uint8_t *qI, const float *w, const uint8_t *kI, const i
     return fail(CSA_ERR_WORKSPACE, "csa_index_topk: workspace needs %zu bytes (got %zu)", need,
                 workspace_bytes);
   if (int rc = need_status()) return rc;
-  return launch_index_topk(qI, w, kI, q_pos, d, idx_out, score_out, workspace,
-                           reinterpret_cast<cudaStream_t>(stream));
+  const int rc = launch_index_topk(qI, w, kI, q_pos, d, idx_out, score_out, workspace,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return rc ? rc : debug_check_topk(idx_out, score_out, q_pos, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t csa_index_topk_mx_workspace(const csa_dims *d) {
@@ -301,8 +331,9 @@ int csa_index_topk_mx(const uint8_t *qI, const uint8_t *qI_scales, const float *
     return fail(CSA_ERR_WORKSPACE, "csa_index_topk_mx: workspace needs %zu bytes (got %zu)", need,
                 workspace_bytes);
   if (int rc = need_status()) return rc;
-  return launch_index_mx(qI, qI_scales, w, kI, kI_scales, q_pos, d, idx_out, score_out, workspace,
-                         reinterpret_cast<cudaStream_t>(stream));
+  const int rc = launch_index_mx(qI, qI_scales, w, kI, kI_scales, q_pos, d, idx_out, score_out, workspace,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  return rc ? rc : debug_check_topk(idx_out, score_out, q_pos, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t csa_attend_workspace(const csa_dims *d) { return d ? attend_workspace(d, false) : 0; }
@@ -376,9 +407,10 @@ int csa_decode_step(const float *x_new, const float *z_new, int32_t n_new, const
       ((uintptr_t)idx_out & 3) || ((uintptr_t)score_out & 3) || ((uintptr_t)lse & 3) || !aligned16(workspace))
     return fail(CSA_ERR_INVALID, "csa_decode_step: misaligned buffer");
   if (int rc = need_status()) return rc;
-  return launch_decode_step(x_new, z_new, n_new, kI_new, q, qI, w, q_pos, codes, scales, kI, win_codes, win_scales,
+  const int rc = launch_decode_step(x_new, z_new, n_new, kI_new, q, qI, w, q_pos, codes, scales, kI, win_codes, win_scales,
                             d, idx_out, score_out, out, lse, workspace, workspace_bytes,
                             reinterpret_cast<cudaStream_t>(stream));
+  return rc ? rc : debug_check_topk(idx_out, score_out, q_pos, d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int csa_sync_status(csa_stream_t stream) {
@@ -393,6 +425,8 @@ int csa_sync_status(csa_stream_t stream) {
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_sync_status: %s", cudaGetErrorString(e));
   if (v & STATUS_TIMEOUT) return fail(CSA_ERR_TIMEOUT, "a device-side wait timed out (status 0x%x)", v);
+  if (v & STATUS_CHECK) return fail(CSA_ERR_CHECK, "an output check failed: a top-k list out of order or range "
+                                    "(status 0x%x)", v);
   if (v & (STATUS_BAD_WEIGHT | STATUS_BAD_INDEX | STATUS_BAD_POSITION))
     return fail(CSA_ERR_INVALID, "invalid device data: %s%s%s (status 0x%x)",
                 (v & STATUS_BAD_WEIGHT) ? "indexer weight off its grid or a NaN block scale; " : "",

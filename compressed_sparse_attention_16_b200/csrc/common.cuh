@@ -42,7 +42,12 @@ enum : unsigned {
                             // not finite, or an E8M0 scale of 0xFF)
   STATUS_BAD_INDEX = 4u,    // attention index outside [0, n_entries) other than -1
   STATUS_BAD_POSITION = 8u, // negative query position (treated as position 0 / no entries)
+  STATUS_CHECK = 16u,       // an output check found a top-k list out of order or range
 };
+// Checks each row's top-k list (indices in range and rank order); a violation
+// sets STATUS_CHECK.  Run after every index call in the CSA_CHECK build.
+int launch_check_topk(const int32_t *idx, const float *score, const int32_t *q_pos, const csa_dims *d,
+                      cudaStream_t stream);
 unsigned *status_word_device_ptr();   // address of the status word, current device
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel), so
 // that launches captured into CUDA graphs issue no attribute calls.

@@ -61,7 +61,8 @@ enum {
   CSA_ERR_UNSUPPORTED = -2, /* valid but outside the compiled shape set      */
   CSA_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed          */
   CSA_ERR_TIMEOUT = -4,     /* a device-side bounded wait gave up            */
-  CSA_ERR_WORKSPACE = -5    /* workspace missing or smaller than required    */
+  CSA_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required    */
+  CSA_ERR_CHECK = -6        /* an output check (csa_check_topk, CSA_CHECK build) failed */
 };
 
 /*
@@ -185,6 +186,25 @@ int csa_index_topk_mx(const uint8_t *qI, const uint8_t *qI_scales, const float *
                       const uint8_t *kI_scales, const int32_t *q_pos, const csa_dims *d,
                       int32_t *idx_out, float *score_out, void *workspace, size_t workspace_bytes,
                       csa_stream_t stream);
+
+/*
+ * csa_check_topk -- checks top-k lists on the device (the pages have no
+ * counterpart: a debugging aid).  For each row at position t =
+ * q_pos[row]: the first min(K, n_vis) indices in [0, n_vis), the rest -1;
+ * with score (may be NULL) each listed score finite and >= 0, the list in
+ * rank order (score descending, equal scores by ascending index) and padding
+ * scores 0.  A violation sets a status bit: the next csa_sync_status()
+ * returns CSA_ERR_CHECK.  Nothing traps.  Uses d->B, Tq, K, m, n_entries;
+ * idx int32 [B, Tq, K], score fp32 [B, Tq, K], q_pos int32 [B, Tq].
+ *
+ * csa_check_build -- 1 in the CSA_CHECK build of the library (libcsa_check.so,
+ * built by `python -m compressed_sparse_attention_16_b200.build --check`),
+ * which runs csa_check_topk after every csa_index_topk, csa_index_topk_mx and
+ * csa_decode_step; 0 otherwise.
+ */
+int csa_check_topk(const int32_t *idx, const float *score, const int32_t *q_pos, const csa_dims *d,
+                   csa_stream_t stream);
+int csa_check_build(void);
 
 /*
  * csa_index_topk_noalloc -- csa_index_topk without a caller-provided workspace.
