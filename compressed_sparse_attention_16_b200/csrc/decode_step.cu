@@ -919,7 +919,37 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       }
     }
   }
-  grid_sync(ws.bar, G, misc, a.status);             // barrier 5: selections and appended rows visible
+  // barrier 5: selections and appended rows visible.  While the other CTAs
+  // finish their selection, the unit's Q goes from its staging buffer into
+  // TMEM (the scan's accumulators are done with): warps 4-7, one head row per
+  // thread; d-block k of the buffer holds d = 16 k .. 16 k + 15, and 32 TMEM
+  // columns take 4 d-blocks (two bf16 per column)
+  tc::fence_before_sync();
+  __syncthreads();
+  if (tid == 0) gb_arrive(ws.bar, misc);
+  if (attB && nloc > 0 && warp >= 4 && warp < 8) {
+    const int h = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const bool qok = uniform(bwait(&bar[BAR_Q], 0, misc, a.status));
+#pragma unroll 1
+    for (int cb = 0; cb < 8 && qok; ++cb) {
+      uint32_t v[32];
+#pragma unroll
+      for (int db = 0; db < 4; ++db) {
+        const uint4 *q4 = reinterpret_cast<const uint4 *>(smem + B_Q + ((cb * 4 + db) * TH + h) * 32);
+        const uint4 x0 = q4[0], x1 = q4[1];
+        v[db * 8 + 0] = x0.x; v[db * 8 + 1] = x0.y; v[db * 8 + 2] = x0.z; v[db * 8 + 3] = x0.w;
+        v[db * 8 + 4] = x1.x; v[db * 8 + 5] = x1.y; v[db * 8 + 6] = x1.z; v[db * 8 + 7] = x1.w;
+      }
+      tc::tmem_st32(misc->tmem + lane_off + TCOL_Q + cb * 32, v);
+    }
+    tc::tmem_wait_st();
+    tc::fence_before_sync();
+    tc::mbar_arrive(&bar[BAR_QT]);
+  }
+  if (tid == 0) gb_wait(ws.bar, G, misc, a.status);
+  __syncthreads();
+  tc::fence_after_sync();
 
   // ---------------------------------------------------------------- B attend
   int *sel = reinterpret_cast<int *>(smem + B_SEL);
@@ -973,29 +1003,8 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         scr[r] = u < n_items ? __ldcg(scp) : 0.f;
       }
       if (c == 0) {
-        if (soft) {
-          // Q row h into TMEM while the gathers are in flight: d-block k of the
-          // staging buffer holds d = 16 k .. 16 k + 15; 32 TMEM columns take 4
-          // d-blocks (two bf16 per column)
-          const bool qok = uniform(bwait(&bar[BAR_Q], 0, misc, a.status));
-#pragma unroll 1
-          for (int cb = 0; cb < 8 && qok; ++cb) {
-            uint32_t v[32];
-#pragma unroll
-            for (int db = 0; db < 4; ++db) {
-              const uint4 *q4 = reinterpret_cast<const uint4 *>(smem + B_Q + ((cb * 4 + db) * TH + h) * 32);
-              const uint4 x0 = q4[0], x1 = q4[1];
-              v[db * 8 + 0] = x0.x; v[db * 8 + 1] = x0.y; v[db * 8 + 2] = x0.z; v[db * 8 + 3] = x0.w;
-              v[db * 8 + 4] = x1.x; v[db * 8 + 5] = x1.y; v[db * 8 + 6] = x1.z; v[db * 8 + 7] = x1.w;
-            }
-            tc::tmem_st32(tbase + lane_off + TCOL_Q + cb * 32, v);
-          }
-          tc::tmem_wait_st();
-          tc::fence_before_sync();
-          tc::mbar_arrive(&bar[BAR_QT]);
-          if (!qok) ok_b = false;
-        }
-        // the tile overlays the Q staging buffer: every head must be copied
+        // Q is in TMEM (moved during barrier 5); the tile overlays its
+        // staging buffer, so every head must have been copied
         if (!uniform(bwait(&bar[BAR_QT], 0, misc, a.status) && ok_b)) { ok_b = false; break; }
       } else if (!uniform(bwait(&bar[BAR_KV_FREE], (c - 1) & 1, misc, a.status))) {
         ok_b = false;

@@ -60,7 +60,7 @@ def _run_chain(B, T0, steps, *, K=512, W=128, HI=4, n_new=4, m=4, seed=0, pass_k
     ind = synth.indexer_inputs(B, steps, N, HI, dI, seed, device="cuda")
     kI_all = ind.kI if kI_override is None else kI_override
     qs = synth.queries(B, steps, H, D, q_scale, seed, device="cuda")
-    st = pipeline.DecodeState(B, D, H, m, W, entry_cap=N, K=K, HI=HI, dI=dI, win_cap=win_cap)
+    st = pipeline.DecodeState(B, D, H, m, W, entry_cap=N, K=K, HI=HI, dI=dI, win_cap=win_cap, fused=True)
     st.prefill_context(x, z, T0, kI=kI_all)
     if not pass_keys:
         st.kI.copy_(kI_all)
@@ -131,7 +131,7 @@ def test_bit_identical_to_separate_calls():
     x, z = synth.tokens(B, Ttot, D, 12, device="cuda")
     ind = synth.indexer_inputs(B, steps, N, 4, 64, 12, device="cuda")
     qs = synth.queries(B, steps, H, D, 512 ** -0.5, 12, device="cuda")
-    a = pipeline.DecodeState(B, D, H, m, 128, entry_cap=N, K=512)
+    a = pipeline.DecodeState(B, D, H, m, 128, entry_cap=N, K=512, fused=True)
     b = pipeline.DecodeState(B, D, H, m, 128, entry_cap=N, K=512, fused=False)
     for st in (a, b):
         st.prefill_context(x, z, T0, kI=ind.kI)
@@ -166,7 +166,7 @@ def test_misaligned_position_is_reported():
     the status word reports it; the context stays usable."""
     B, D, H, m = 1, 512, 128, 4
     N = 64
-    st = pipeline.DecodeState(B, D, H, m, 16, entry_cap=N, K=8)
+    st = pipeline.DecodeState(B, D, H, m, 16, entry_cap=N, K=8, fused=True)
     x, z = synth.tokens(B, 4, D, 0, device="cuda")
     ind = synth.indexer_inputs(B, 1, N, 4, 64, 0, device="cuda")
     q = synth.queries(B, 1, H, D, 0.05, 0, device="cuda")
