@@ -60,8 +60,8 @@ def op_work(wl):
         n_new = 4 if wl.kind != "hca_decode" else m
         N = wl.N
         raw = B * n_new * D * 8
-        w["compress_entry"] = dict(bytes=raw + B * (n_new // m) * ent, flops=0)
-        w["compress_window"] = dict(bytes=raw + B * n_new * ent, flops=0)
+        # entries and window in one pass over the new tokens (x and z once)
+        w["compress"] = dict(bytes=raw + B * (n_new // m) * ent + B * n_new * ent, flops=0)
         if wl.kind == "hca_decode":
             items = N + W
             w["hca_attend"] = dict(bytes=B * items * ent + 2 * B * H * D * 2 + B * H * 4,
@@ -79,8 +79,7 @@ def op_work(wl):
                                     flops=sum(v["flops"] for v in w.values()), aggregate=True)
     else:   # prefill
         T, N = wl.T, wl.N
-        w["compress_entry"] = dict(bytes=B * T * D * 8 + B * N * ent, flops=0)
-        w["compress_window"] = dict(bytes=B * T * D * 8 + B * T * ent, flops=0)
+        w["compress"] = dict(bytes=B * T * D * 8 + B * N * ent + B * T * ent, flops=0)
         pairs = B * sum_visible(T, m, N)
         w["index_topk"] = dict(bytes=B * N * (wl.dI // 2) + B * T * (wl.HI * (wl.dI // 2 + 4) + K * 8),
                                flops=2.0 * pairs * wl.HI * wl.dI)
@@ -276,8 +275,7 @@ class Runner:
             z = self.z if inputs is None else inputs["z"]
             q = self.q if inputs is None else inputs["q"]
             return [
-                ("compress_entry", lambda: csa.compress(x, z, wl.m, self.codes, self.scales)),
-                ("compress_window", lambda: csa.compress(x, z, 1, self.wcodes, self.wscales)),
+                ("compress", lambda: csa.compress_ew(x, z, wl.m, self.codes, self.scales, self.wcodes, self.wscales)),
                 ("index_topk", lambda: csa.index_topk(self.ind.qI, self.ind.w, self.ind.kI, self.q_pos, self.dims,
                                                       self.idx, self.score, workspace=self.ws_i)),
                 ("attend", lambda: csa.attend(q, self.codes, self.scales, self.idx, self.wcodes, self.wscales,
@@ -294,10 +292,9 @@ class Runner:
             src, first = (inputs["x"], inputs["z"]), 0
         q = self.q if inputs is None else inputs["q"]
         out = [
-            ("compress_entry", lambda: csa.compress(src[0], src[1], wl.m, st.codes, st.scales, dst_first=t0 // wl.m,
-                                                    T=self.n_new, first_token=first)),
-            ("compress_window", lambda: csa.compress(src[0], src[1], 1, st.win_codes, st.win_scales, dst_first=t0,
-                                                     ring_cap=st.win_cap, T=self.n_new, first_token=first)),
+            ("compress", lambda: csa.compress_ew(src[0], src[1], wl.m, st.codes, st.scales, st.win_codes, st.win_scales,
+                                                 dst_first=t0 // wl.m, win_first=t0, win_ring_cap=st.win_cap,
+                                                 T=self.n_new, first_token=first)),
         ]
         if wl.kind == "hca_decode":
             ws = self._ws(csa.attend_workspace(d, True), "_ws_hca")

@@ -30,6 +30,7 @@ CSA_ERR_CHECK = -6
 # every symbol declared in include/csa.h
 SYMBOLS = (
     "csa_compress",
+    "csa_compress_ew",
     "csa_index_topk_workspace",
     "csa_index_topk",
     "csa_index_topk_noalloc",
@@ -94,6 +95,9 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     L.csa_compress.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _I64, _I64, _I32, _P, _P]
     L.csa_compress.restype = ctypes.c_int
+    L.csa_compress_ew.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _I64, _P, _P, _I64, _I64, _I32, _P, _P, _I64,
+                                  _I64, _I32, _P, _P]
+    L.csa_compress_ew.restype = ctypes.c_int
     L.csa_index_topk_workspace.argtypes = [ctypes.POINTER(Dims)]
     L.csa_index_topk_workspace.restype = _SZ
     L.csa_index_topk.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Dims), _P, _P, _P, _SZ, _P]
@@ -191,6 +195,33 @@ def compress(x: torch.Tensor, z: torch.Tensor, m: int, codes: torch.Tensor, scal
                               _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
                               dst_first, codes.shape[1], ring_cap,
                               _ptr(pooled, torch.float32, "pooled", dev), _stream(stream)))
+
+
+def compress_ew(x: torch.Tensor, z: torch.Tensor, m: int, codes: torch.Tensor, scales: torch.Tensor,
+                win_codes: torch.Tensor, win_scales: torch.Tensor, dst_first: int = 0, ring_cap: int = 0,
+                win_first: int = 0, win_ring_cap: int = 0, pooled: torch.Tensor | None = None,
+                T: int | None = None, first_token: int = 0, stream=None) -> None:
+    """csa_compress_ew: the m-token entries of tokens [first_token, first_token + T)
+    of x, z [B, Ttot, D] (as compress) and every one of those tokens as a
+    window entry (compress with m = 1), in one pass."""
+    if x.dim() != 3 or z.shape != x.shape:
+        raise ValueError("x and z must be [B, T, D] of equal shape")
+    B, Ttot, D = x.shape
+    T = Ttot - first_token if T is None else T
+    if first_token < 0 or first_token + T > Ttot:
+        raise ValueError("token range outside x")
+    for c, s_, what in ((codes, scales, "codes"), (win_codes, win_scales, "win_codes")):
+        if c.dim() != 3 or c.shape[0] != B or c.shape[2] != D or s_.shape != c.shape[:2]:
+            raise ValueError(f"{what} must be [B, cap, D] with scales [B, cap]")
+    dev = x.device
+    off = first_token * D * 4
+    _check(lib().csa_compress_ew(_ptr(x, torch.float32, "x") + off, _ptr(z, torch.float32, "z", dev) + off, B, T, D,
+                                 m, Ttot * D,
+                                 _ptr(codes, torch.uint8, "codes", dev), _ptr(scales, torch.float32, "scales", dev),
+                                 dst_first, codes.shape[1], ring_cap,
+                                 _ptr(win_codes, torch.uint8, "win_codes", dev),
+                                 _ptr(win_scales, torch.float32, "win_scales", dev), win_first, win_codes.shape[1],
+                                 win_ring_cap, _ptr(pooled, torch.float32, "pooled", dev), _stream(stream)))
 
 
 def quantize_mxfp4(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:

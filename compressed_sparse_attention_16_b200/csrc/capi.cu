@@ -11,6 +11,10 @@
 
 namespace csa {
 
+int launch_compress_ew(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride, uint8_t *codes,
+                       float *scales, int64_t dst_first, int64_t dst_bstride, int ring_cap, uint8_t *wcodes,
+                       float *wscales, int64_t w_first, int64_t w_bstride, int w_ring, float *pooled,
+                       cudaStream_t stream);
 int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
                     uint8_t *codes, float *scales, int64_t dst_first, int64_t dst_bstride,
                     int ring_cap, float *pooled, cudaStream_t stream);
@@ -279,6 +283,38 @@ int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D
     return fail(CSA_ERR_INVALID, "csa_compress: dst_batch_stride < ring_cap");
   return launch_compress(x, z, B, T, D, m, x_batch_stride, codes, scales, dst_first,
                          dst_batch_stride, ring_cap, pooled, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int csa_compress_ew(const float *x, const float *z, int32_t B, int32_t T, int32_t D, int32_t m,
+                    int64_t x_batch_stride, uint8_t *codes, float *scales, int64_t dst_first,
+                    int64_t dst_batch_stride, int32_t ring_cap, uint8_t *win_codes, float *win_scales,
+                    int64_t win_first, int64_t win_batch_stride, int32_t win_ring_cap, float *pooled,
+                    csa_stream_t stream) {
+  clear_error();
+  if (B < 0 || T < 0 || m < 1) return fail(CSA_ERR_INVALID, "csa_compress_ew: bad B/T/m (%d/%d/%d)", B, T, m);
+  if (D < 4 || D > 1024 || D % 4 || !pow2(D / 4))
+    return fail(CSA_ERR_UNSUPPORTED, "csa_compress_ew: D=%d (needs D/4 a power of two, 4..1024)", D);
+  if (B == 0 || T == 0) return CSA_OK;
+  if (!x || !z || !codes || !scales || !win_codes || !win_scales)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: NULL buffer");
+  if (!aligned16(x) || !aligned16(z) || (pooled && !aligned16(pooled)) || ((uintptr_t)codes & 3) ||
+      ((uintptr_t)win_codes & 3))
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: misaligned buffer");
+  if (x_batch_stride % 4 || (B > 1 && x_batch_stride < (int64_t)T * D))
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: x_batch_stride must be a multiple of 4 and >= T*D");
+  if (dst_first < 0 || ring_cap < 0 || win_first < 0 || win_ring_cap < 0)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: negative first slot or ring capacity");
+  if (ring_cap == 0 && B > 1 && dst_batch_stride < dst_first + T / m)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: dst_batch_stride too small");
+  if (ring_cap > 0 && B > 1 && dst_batch_stride < ring_cap)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: dst_batch_stride < ring_cap");
+  if (win_ring_cap == 0 && B > 1 && win_batch_stride < win_first + T)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: win_batch_stride too small");
+  if (win_ring_cap > 0 && B > 1 && win_batch_stride < win_ring_cap)
+    return fail(CSA_ERR_INVALID, "csa_compress_ew: win_batch_stride < win_ring_cap");
+  return launch_compress_ew(x, z, B, T, D, m, x_batch_stride, codes, scales, dst_first, dst_batch_stride, ring_cap,
+                            win_codes, win_scales, win_first, win_batch_stride, win_ring_cap, pooled,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t csa_index_topk_workspace(const csa_dims *d) {

@@ -216,7 +216,160 @@ compress_tokens_kernel(const float *__restrict__ x, const float *__restrict__ z,
   }
 }
 
+// Entries and window in one pass: each group of D/4 threads pools one block
+// of m tokens (m = 2, 4 or 8) into an entry exactly as compress_kernel does,
+// and also quantises each of the block's m tokens on its own as a window
+// entry (the one-token case of the same rule: C = x, s = amax / 448).  The
+// block's tokens are read once; the m + 1 amax reductions run together.
+// Instantiated for m = 2, 4 and 8 (M).
+constexpr int kMaxEwM = 8;
+
+template <int M>
+__global__ void __launch_bounds__(kThreads)
+compress_ew_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_per_seq, int64_t n_total,
+                   int D, int T, int64_t x_bstride, uint8_t *__restrict__ codes, float *__restrict__ scales,
+                   int64_t dst_first, int64_t dst_bstride, int ring_cap, uint8_t *__restrict__ wcodes,
+                   float *__restrict__ wscales, int64_t w_first, int64_t w_bstride, int w_ring,
+                   float *__restrict__ pooled) {
+  constexpr int m = M;
+  __shared__ float red[kThreads / 32][M + 1];
+  const int L = D >> 2;
+  const int groups = kThreads / L;
+  const int g = threadIdx.x / L;
+  const int lane = threadIdx.x - g * L;
+  const int64_t e = (int64_t)blockIdx.x * groups + g;
+  int64_t b = 0, i = 0;
+  const bool valid = g < groups && e < n_total;
+  if (valid) {
+    b = e / n_per_seq;
+    i = e - b * n_per_seq;
+  }
+  const bool write_entry = valid && !(ring_cap > 0 && i + ring_cap < n_per_seq);
+  float4 xv[M];
+  float C[4] = {0.f, 0.f, 0.f, 0.f};
+  float v[M + 1];
+#pragma unroll
+  for (int u = 0; u <= M; ++u) v[u] = 0.f;
+  if (valid) {
+    const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + lane;
+    const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + lane;
+    float4 zv[M];
+#pragma unroll
+    for (int u = 0; u < M; ++u) {
+      xv[u] = __ldg(xp + (int64_t)u * L);
+      zv[u] = __ldg(zp + (int64_t)u * L);
+    }
+    OnlineSoftmax4 sm;
+    sm.init();
+#pragma unroll
+    for (int u = 0; u < M; ++u) sm.push(xv[u], zv[u]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) C[c] = __fdiv_rn(sm.acc[c], sm.l[c]);
+    v[0] = fmaxf(fmaxf(fabsf(C[0]), fabsf(C[1])), fmaxf(fabsf(C[2]), fabsf(C[3])));
+#pragma unroll
+    for (int u = 0; u < M; ++u)
+      v[u + 1] = fmaxf(fmaxf(fabsf(xv[u].x), fabsf(xv[u].y)), fmaxf(fabsf(xv[u].z), fabsf(xv[u].w)));
+  }
+  // the m + 1 maxima over the group's L threads
+  const int width = L < 32 ? L : 32;
+#pragma unroll
+  for (int u = 0; u <= M; ++u)
+    for (int o = width >> 1; o > 0; o >>= 1) v[u] = fmaxf(v[u], __shfl_xor_sync(0xffffffffu, v[u], o));
+  if (L > 32) {
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+      for (int u = 0; u <= M; ++u) red[warp][u] = v[u];
+    }
+    __syncthreads();
+    const int w0 = (g * L) >> 5, nw = L >> 5;
+#pragma unroll
+    for (int u = 0; u <= M; ++u) {
+      float a = 0.f;
+      for (int k = 0; k < nw; ++k) a = fmaxf(a, red[w0 + k][u]);
+      v[u] = a;
+    }
+  }
+  if (!valid) return;
+  auto quant = [&](const float (&c)[4], float a, uint32_t &word) {
+    float s = __fdiv_rn(a, 448.f);
+    if (!(s > 0.f)) s = 1.f;
+    word = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t q = __nv_cvt_float_to_fp8(__fdiv_rn(c[k], s), __NV_SATFINITE, __NV_E4M3);
+      word |= q << (8 * k);
+    }
+    return s;
+  };
+  if (write_entry) {
+    uint32_t word;
+    const float s = quant(C, v[0], word);
+    int64_t slot = dst_first + i;
+    if (ring_cap > 0) slot %= ring_cap;
+    const int64_t ent = b * dst_bstride + slot;
+    reinterpret_cast<uint32_t *>(codes + ent * D)[lane] = word;
+    if (lane == 0) scales[ent] = s;
+  }
+  if (pooled)
+    reinterpret_cast<float4 *>(pooled + (b * n_per_seq + i) * (int64_t)D)[lane] = make_float4(C[0], C[1], C[2], C[3]);
+#pragma unroll
+  for (int u = 0; u < M; ++u) {
+    const int64_t p = i * m + u;                      // token of the call
+    if (w_ring > 0 && p + w_ring < T) continue;
+    const float c4[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+    uint32_t word;
+    const float s = quant(c4, v[u + 1], word);
+    int64_t slot = w_first + p;
+    if (w_ring > 0) slot %= w_ring;
+    const int64_t ent = b * w_bstride + slot;
+    reinterpret_cast<uint32_t *>(wcodes + ent * D)[lane] = word;
+    if (lane == 0) wscales[ent] = s;
+  }
+}
+
 }  // namespace
+
+int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
+                    uint8_t *codes, float *scales, int64_t dst_first, int64_t dst_bstride,
+                    int ring_cap, float *pooled, cudaStream_t stream);
+
+int launch_compress_ew(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride, uint8_t *codes,
+                       float *scales, int64_t dst_first, int64_t dst_bstride, int ring_cap, uint8_t *wcodes,
+                       float *wscales, int64_t w_first, int64_t w_bstride, int w_ring, float *pooled,
+                       cudaStream_t stream) {
+  const int L = D / 4;
+  const int n = T / m;
+  if ((m != 2 && m != 4 && m != 8) || L > kThreads || n == 0) {
+    // not fused: the entries, then every token as a window entry
+    if (int rc = launch_compress(x, z, B, T, D, m, x_bstride, codes, scales, dst_first, dst_bstride, ring_cap,
+                                 pooled, stream))
+      return rc;
+    return launch_compress(x, z, B, T, D, 1, x_bstride, wcodes, wscales, w_first, w_bstride, w_ring, nullptr,
+                           stream);
+  }
+  const int64_t total = (int64_t)B * n;
+  const int groups = kThreads / L;
+  const int64_t grid = (total + groups - 1) / groups;
+  if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_ew: too many entries");
+#define CSA_EW(M_)                                                                                       \
+  compress_ew_kernel<M_><<<(unsigned)grid, kThreads, 0, stream>>>(x, z, n, total, D, T, x_bstride, codes, scales, \
+                                                                  dst_first, dst_bstride, ring_cap, wcodes,       \
+                                                                  wscales, w_first, w_bstride, w_ring, pooled)
+  if (m == 2) CSA_EW(2);
+  else if (m == 4) CSA_EW(4);
+  else CSA_EW(8);
+#undef CSA_EW
+  count_launches(1);
+  if (int rc = check_launch("compress_ew_kernel")) return rc;
+  const int tail = T - n * m;                         // tokens past the last full block: window only
+  if (tail == 0) return CSA_OK;
+  // tokens [n m, T) of each sequence: the call's tokens n m .. T - 1 (the ring
+  // keeps the same ones: token n m + j is skipped iff j + w_ring < tail)
+  const int64_t off = (int64_t)n * m * D;
+  return launch_compress(x + off, z + off, B, tail, D, 1, x_bstride, wcodes, wscales, w_first + (int64_t)n * m,
+                         w_bstride, w_ring, nullptr, stream);
+}
 
 int launch_compress(const float *x, const float *z, int B, int T, int D, int m, int64_t x_bstride,
                     uint8_t *codes, float *scales, int64_t dst_first, int64_t dst_bstride,

@@ -19,8 +19,8 @@ import dataclasses
 
 import torch
 
-from . import (Dims, attend, attend_workspace, compress, decode_step, decode_step_workspace, hca_attend, index_topk,
-               index_topk_workspace)
+from . import (Dims, attend, attend_workspace, compress, compress_ew, decode_step, decode_step_workspace, hca_attend,
+               index_topk, index_topk_workspace)
 
 
 def prefer_fused_step(B: int, device=None) -> bool:
@@ -65,8 +65,7 @@ def prefill(x, z, q, qI, w, kI, *, m: int, K: int, W: int, softmax_scale: float 
     scales = torch.empty((B, N), dtype=torch.float32, device=dev)
     win_codes = torch.empty((B, T, D), dtype=torch.uint8, device=dev)
     win_scales = torch.empty((B, T), dtype=torch.float32, device=dev)
-    compress(x, z, m, codes, scales, pooled=pooled)
-    compress(x, z, 1, win_codes, win_scales)
+    compress_ew(x, z, m, codes, scales, win_codes, win_scales, pooled=pooled)
     q_pos = torch.arange(T, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
     dims = Dims(B=B, Tq=T, H=H, D=D, HI=HI, dI=dI, K=K, W=W, m=m, n_entries=N, entry_cap=N,
                 win_cap=T, softmax_scale=softmax_scale)
@@ -163,9 +162,8 @@ class DecodeState:
         assert self.n_tokens % self.m == 0 and n % self.m == 0
         first = self.n_entries
         assert first + n // self.m <= self.entry_cap
-        compress(x_new, z_new, self.m, self.codes, self.scales, dst_first=first)
-        compress(x_new, z_new, 1, self.win_codes, self.win_scales, dst_first=self.n_tokens,
-                 ring_cap=self.win_cap)
+        compress_ew(x_new, z_new, self.m, self.codes, self.scales, self.win_codes, self.win_scales,
+                    dst_first=first, win_first=self.n_tokens, win_ring_cap=self.win_cap)
         if kI_new is not None and self.kI is not None:
             self.kI[:, first:first + n // self.m].copy_(kI_new)
         self.n_tokens += n
@@ -231,9 +229,8 @@ class DecodeState:
             self.kI[:, first:first + n // self.m].copy_(kI_new)
         side.wait_stream(main)
         with torch.cuda.stream(side):
-            compress(x_new, z_new, self.m, self.codes, self.scales, dst_first=first)
-            compress(x_new, z_new, 1, self.win_codes, self.win_scales, dst_first=self.n_tokens,
-                     ring_cap=self.win_cap)
+            compress_ew(x_new, z_new, self.m, self.codes, self.scales, self.win_codes, self.win_scales,
+                        dst_first=first, win_first=self.n_tokens, win_ring_cap=self.win_cap)
         x_new.record_stream(side)
         z_new.record_stream(side)
         self.n_tokens += n

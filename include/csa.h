@@ -118,6 +118,24 @@ int csa_compress(const float *x, const float *z, int32_t B, int32_t T, int32_t D
                  csa_stream_t stream);
 
 /*
+ * csa_compress_ew -- csa_compress for the entries and, in the same pass over
+ * x, every one of the T tokens as a window entry (csa_compress with m = 1):
+ * the block's tokens are read once.  Arguments as csa_compress, plus the
+ * window's codes u8 [B, win_cap, D] and scales fp32 [B, win_cap] (batch
+ * stride win_batch_stride entries), first slot win_first and ring capacity
+ * win_ring_cap (0: no ring; with a ring only the call's last win_ring_cap
+ * tokens are written, token p at slot (win_first + p) mod win_ring_cap).
+ * Results are bit-identical to the two csa_compress calls.  Fused for
+ * m = 2, 4 or 8 and D <= 1024; other m run the two passes.  Tokens past the
+ * last full block enter the window only.
+ */
+int csa_compress_ew(const float *x, const float *z, int32_t B, int32_t T, int32_t D, int32_t m,
+                    int64_t x_batch_stride, uint8_t *codes, float *scales, int64_t dst_first,
+                    int64_t dst_batch_stride, int32_t ring_cap, uint8_t *win_codes, float *win_scales,
+                    int64_t win_first, int64_t win_batch_stride, int32_t win_ring_cap, float *pooled,
+                    csa_stream_t stream);
+
+/*
  * csa_index_topk -- Lightning-Indexer scores and top-k.
  * (jiwasawa "Compressed Sparse Attention (CSA)": indexer scores per query and
  *  a top-k selector; hazakura.dev "衝撃1": FP4 indexer; studioglobal.ai

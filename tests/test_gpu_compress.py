@@ -106,3 +106,48 @@ def test_compress_full_hca_config_sampled():
         parity.check_codes(codes[b, bl].cpu().numpy(), scales[b, bl].cpu().numpy(), ref, A)
     del x, z
     torch.cuda.empty_cache()
+
+
+def _ew_pair(B, T, D, m, cap, wcap, dst_first=0, ring=0, win_first=0, win_ring=0, seed=0, pooled=False):
+    """csa_compress_ew against csa_compress (entries) + csa_compress with m = 1
+    (window), on sentinel-filled outputs: every byte equal."""
+    x, z = synth.tokens(B, T, D, seed, device="cuda")
+    outs = []
+    for fused in (True, False):
+        codes = torch.full((B, cap, D), 0xA5, dtype=torch.uint8, device="cuda")
+        scales = torch.full((B, cap), -3.0, device="cuda")
+        wc = torch.full((B, wcap, D), 0x5A, dtype=torch.uint8, device="cuda")
+        ws = torch.full((B, wcap), -5.0, device="cuda")
+        pl = torch.full((B, T // m, D), -7.0, device="cuda") if pooled else None
+        if fused:
+            csa.compress_ew(x, z, m, codes, scales, wc, ws, dst_first=dst_first, ring_cap=ring, win_first=win_first,
+                            win_ring_cap=win_ring, pooled=pl)
+        else:
+            csa.compress(x, z, m, codes, scales, dst_first=dst_first, ring_cap=ring, pooled=pl)
+            csa.compress(x, z, 1, wc, ws, dst_first=win_first, ring_cap=win_ring)
+        csa.sync_status()
+        outs.append([t.cpu() for t in (codes, scales, wc, ws) + ((pl,) if pooled else ())])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B,T,D,m", [(2, 1030, 512, 4), (3, 64, 64, 2), (1, 96, 1024, 8), (2, 40, 128, 4)])
+def test_compress_ew_equals_two_passes(B, T, D, m):
+    """Entries and window in one pass: bit-identical to the two calls, with a
+    ragged tail of tokens that enter only the window, and the pooled output."""
+    _ew_pair(B, T, D, m, cap=T // m + 3, wcap=T + 2, seed=B * 7 + m, pooled=True)
+
+
+def test_compress_ew_rings_and_offsets():
+    """Decode-style appends: entries at an offset, the window as a ring that
+    wraps, and a window ring smaller than the call (only its last tokens
+    survive)."""
+    _ew_pair(3, 8, 512, 4, cap=200, wcap=16, dst_first=100, win_first=30, win_ring=16, seed=1)
+    _ew_pair(2, 12, 512, 4, cap=40, wcap=5, dst_first=7, win_first=3, win_ring=5, seed=2)
+    _ew_pair(2, 16, 512, 4, cap=3, wcap=64, dst_first=1, ring=3, win_first=0, seed=3)   # entry ring too
+
+
+@pytest.mark.parametrize("m", [1, 16])
+def test_compress_ew_unfused_shapes(m):
+    """m outside the fused range runs the two passes inside the call."""
+    _ew_pair(2, 64, 512, m, cap=64 // m + 1, wcap=70, seed=m)
