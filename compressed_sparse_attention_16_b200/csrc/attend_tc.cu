@@ -12,7 +12,7 @@
 // Work split: one CTA per (query row, half of D, item split).  With M = 128
 // query heads, S = Q K^T (K = 512) lands in TMEM with one head per lane; the
 // output half O[:, dh*256 : dh*256+256] = P V accumulates in 256 TMEM columns
-// across the CTA's chunks of 32 items.  Both halves of a row compute the same
+// across the CTA's chunks of 64 items.  Both halves of a row compute the same
 // S (each needs the full 512-wide dot products) and keep bit-identical softmax
 // state, so their halves combine without exchange.  The item splits of one
 // (row, half) (1, 2, 4 or 8) form a thread-block cluster: each CTA writes its
@@ -20,18 +20,27 @@
 // hardware cluster barrier orders them, and CTA c then combines the final
 // rows of heads [c * 128 / S, +128 / S):
 //   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
-// Q arrives by 32 TMA boxes of 128 heads x 16 d (32-byte swizzle, the layout
-// the MMA reads); the CTA's gathered rows are prefetched into L2 right after
-// the selection is compacted.
+//
+// Tensor memory (512 columns): O (256), S double-buffered (2 x 64), and the
+// first half of Q (d < 256, 128 columns of bf16 pairs) as the A operand of
+// the first 16 QK MMAs; the second half of Q stays in shared memory (16 TMA
+// boxes of 128 heads x 16 d, 32-byte swizzle).  That frees the room for two
+// 64-item tiles, so the loaders fill one tile while the tensor core reads the
+// other.  P (bf16) overwrites the first 32 columns of its S buffer and is the
+// TMEM A operand of the PV MMAs, so it never touches shared memory.  A
+// tcgen05 MMA with M = 128 and K = 16 costs about the same for N = 32 and
+// N = 64 (about 50 cycles, its issue floor, against 135 at N = 256), so the
+// QK product runs at N = 64.
 //
 // Roles (288 threads):
-//   warps 0-3  gather 32 items per chunk, convert E4M3 codes exactly to bf16
+//   warps 0-3  gather 64 items per chunk (dense lists: one bulk L2 prefetch
+//              of the chunk two ahead), convert E4M3 codes exactly to bf16
 //              and store them in the "core matrix" layout (8 rows x 16 B);
-//   warps 4-7  Q to shared memory (while the first chunks are gathered), then
-//              softmax: one head per thread, lazy rescaling of O (only when a
-//              chunk raises the running max by more than 2^8), P = p * scale
-//              written to shared memory;
-//   warp 8     TMEM allocation and the single MMA-issuing thread.
+//   warps 4-7  first half of Q into TMEM, then softmax: one head per thread,
+//              lazy rescaling of O (only when a chunk raises the running max
+//              by more than 2^8), P = p * scale written to TMEM;
+//   warp 8     TMEM allocation, the Q TMA, and the single MMA-issuing thread,
+//              which issues whichever of PV(c) and QK(c + 2) is ready first.
 // Item scales multiply the logits and P, never the codes, so the bf16 tiles
 // hold the E4M3 values exactly.  Every mbarrier wait is bounded by wall time;
 // on expiry the CTA sets the library's status word and unwinds.
@@ -43,33 +52,48 @@ namespace {
 
 constexpr int TH = 128;          // heads = MMA M
 constexpr int TD = 512;          // entry width
-constexpr int CH = 32;           // items per chunk = QK MMA N
 constexpr int DHALF = 256;       // output columns per CTA = PV MMA N
+constexpr int CH = 64;           // items per chunk = QK MMA N
+constexpr uint32_t GS = CH * 16; // byte step between d-groups of a KV tile
 constexpr int kThreads = 288;
 constexpr int kMaxSel = 2048;
+constexpr int kPrefetchAhead = 2;  // chunks
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.f;
 constexpr unsigned long long kWaitNs = 2000000000ull;   // 2 s per wait
 
-// shared memory map (bytes)
-constexpr uint32_t OFF_Q = 0;                              // 128 x 512 bf16 = 128 KiB
-constexpr uint32_t OFF_KV = OFF_Q + TH * TD * 2;           // 2 x (32 x 512 bf16) = 64 KiB
-constexpr uint32_t KV_BYTES = CH * TD * 2;
-constexpr uint32_t OFF_P = OFF_KV + 2 * KV_BYTES;          // 2 x (128 x 32 bf16) = 16 KiB
-constexpr uint32_t P_BYTES = TH * CH * 2;
-constexpr uint32_t OFF_SEL = OFF_P + 2 * P_BYTES;          // int32 [2048]
-constexpr uint32_t OFF_SCALE = OFF_SEL + kMaxSel * 4;      // fp32 [2][32]
-constexpr uint32_t OFF_BAR = OFF_SCALE + 2 * CH * 4;       // mbarriers
-constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 64;
+// Shared memory map (bytes):
+//   QH    128 heads x d 256..511 bf16 = 64 KiB (16 boxes of 4 KiB)
+//   KV    2 x (64 x 512 bf16) = 128 KiB
+//   SEL   int32 [2048] (sparse instances only)
+//   SCALE fp32 [2][64] item scales (for P) and [2][64] scales x softmax
+//         scale x log2(e) (for the logits)
+template <bool SEL>
+struct Lay {
+  static constexpr uint32_t OFF_QH = 0;
+  static constexpr uint32_t OFF_KV = OFF_QH + TH * (TD / 2) * 2;
+  static constexpr uint32_t KV_BYTES = CH * TD * 2;
+  static constexpr uint32_t OFF_SEL = OFF_KV + 2 * KV_BYTES;
+  static constexpr uint32_t OFF_SCALE = OFF_SEL + (SEL ? kMaxSel * 4 : 0);
+  static constexpr uint32_t OFF_BAR = OFF_SCALE + 2 * 2 * CH * 4;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 64;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
 
 // TMEM columns
-constexpr uint32_t TCOL_O = 0;        // 256 columns
-constexpr uint32_t TCOL_S = 256;      // 2 x 32 columns
+constexpr uint32_t TCOL_O = 0;        // 256
+constexpr uint32_t TCOL_S = 256;      // 2 x 64
+constexpr uint32_t TCOL_QL = 384;     // 128: Q[:, 0:256] as bf16 pairs
 constexpr uint32_t TMEM_COLS = 512;
 
-enum { BAR_KV_FULL = 0, BAR_KV_FREE = 2, BAR_S_FULL = 4, BAR_P_FULL = 6, BAR_PV_DONE = 8, BAR_FIN = 9,
-       BAR_Q = 10 };
+// Each item tile is written in two halves of d: half A (the 256 columns
+// this CTA's PV product does not read, needed only by the QK MMAs over
+// them) and half B (this CTA's output half).  Half A of a slot is free once
+// the QK MMAs over it are done, half B once PV is done, so the loaders
+// refill half A of chunk c + 2 while PV(c) is still pending.
+enum { BAR_FULL_A = 0, BAR_FULL_B = 2, BAR_FREE_A = 4, BAR_FREE_B = 6, BAR_S_FULL = 8, BAR_P_FULL = 10,
+       BAR_PV_DONE = 12, BAR_FIN = 13, BAR_Q = 14, BAR_QT = 15, kNumBars = 16 };
 
 struct Misc {
   uint32_t tmem_base;
@@ -107,32 +131,45 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // Byte offsets in the core-matrix layouts.  g counts 16-byte groups along
-// the contraction-side dimension of each tile (8 bf16).  Every tile keeps
-// the 8-row-group stride at 128 B and the other stride at most 2 KiB, so all
-// descriptor strides stay small.
-//   Q  [128 heads][512 d]:  not core matrices: 32 TMA boxes [128 heads][16 d]
-//                           of 4 KiB with 32-byte swizzle, box k at k * 4096
-//   KV [32 items][512 d]:   g = d/8,     g-stride 512 B,  item-group stride 128 B
-//   P  [128 heads][32 items]: g = item/8, g-stride 2048 B, head-group stride 128 B
-__device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 512 + (i >> 3) * 128 + (i & 7) * 16; }
-__device__ __forceinline__ uint32_t p_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
+// the contraction-side dimension of each tile (8 bf16).
+//   QH [128 heads][256 d]:   not core matrices: 16 TMA boxes [128 heads][16 d]
+//                            of 4 KiB with 32-byte swizzle, box k at k * 4096
+//   KV [64 items][512 d]:    g = d/8,     g-stride 1 KiB,  item-group stride 128 B
+__device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * GS + (i >> 3) * 128 + (i & 7) * 16; }
 
-// 16 E4M3 codes -> 16 bf16 (exact), as two 16-byte words
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, uint4 &lo, uint4 &hi) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 a = e4m3x2_to_float2((uint16_t)(w[k] & 0xFFFF));
-    const float2 b = e4m3x2_to_float2((uint16_t)(w[k] >> 16));
-    const __nv_bfloat162 ab = __float22bfloat162_rn(a);
-    const __nv_bfloat162 bb = __float22bfloat162_rn(b);
-    o[2 * k] = *reinterpret_cast<const uint32_t *>(&ab);
-    o[2 * k + 1] = *reinterpret_cast<const uint32_t *>(&bb);
-  }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
+// packed fp32 pairs (low word first) and the two-lane PTX arithmetic
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+  return v;
 }
+__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32: a few ulp;
+// results below 2^-126 flush to zero, far below what a bf16 P or the fp32
+// row sum can hold next to the row's largest term, which is >= 2^-8)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 
 struct Args {
   const __nv_bfloat16 *q;
@@ -153,13 +190,19 @@ struct Args {
   unsigned *status;
 };
 
+template <bool SEL>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                 const Args a) {
+  using Lt = Lay<SEL>;
+  constexpr uint32_t OFF_QH = Lt::OFF_QH, OFF_KV = Lt::OFF_KV, KV_BYTES = Lt::KV_BYTES;
+  constexpr uint32_t OFF_SEL = Lt::OFF_SEL, OFF_SCALE = Lt::OFF_SCALE;
+  constexpr uint32_t OFF_BAR = Lt::OFF_BAR, OFF_MISC = Lt::OFF_MISC;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   Misc *misc = reinterpret_cast<Misc *>(smem + OFF_MISC);
   int *sel = reinterpret_cast<int *>(smem + OFF_SEL);
-  float *iscale = reinterpret_cast<float *>(smem + OFF_SCALE);
+  float *iscale = reinterpret_cast<float *>(smem + OFF_SCALE);        // [2][CH] item scales
+  float *lscale = iscale + 2 * CH;                                     // [2][CH] logit factors
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x % a.splits;        // == rank in the cluster
@@ -179,15 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
 
   if (tid == 0) {
     misc->abort = 0;
-    for (int i = 0; i < 10; ++i) tc::mbar_init(&bars[i], (i == BAR_KV_FULL || i == BAR_KV_FULL + 1) ? 128
-                                                       : (i == BAR_P_FULL || i == BAR_P_FULL + 1) ? 128 : 1);
-    tc::mbar_init(&bars[BAR_Q], 1);
+    for (int i = 0; i < kNumBars; ++i)
+      tc::mbar_init(&bars[i], (i < BAR_FREE_A || i == BAR_P_FULL || i == BAR_P_FULL + 1 || i == BAR_QT) ? 128 : 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
   if (warp == 8) {
     tc::tmem_alloc(&misc->tmem_base, TMEM_COLS);
-  } else if (a.idx) {
+  } else if (SEL && a.idx) {
     // ordered compaction of the valid selected entries (warps 0-7)
     const int32_t *irow = a.idx + (int64_t)row * a.K;
     int base = 0;
@@ -210,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const int nsel = a.idx ? misc->nsel : nvis;
+  const int nsel = (SEL && a.idx) ? misc->nsel : nvis;
   const int n_items = nsel + nwin;
   const int nch = (n_items + CH - 1) / CH;
   const int c_begin = split * a.cps;
@@ -218,97 +260,181 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   const int nloc = max(0, c_end - c_begin);
   const uint32_t tbase = misc->tmem_base;
   const uint32_t sbase = tc::smem_u32(smem);
-  if (warp == 8) {
-    // Q (32 boxes of 128 heads x 16 d, 32-byte swizzle: box k is the A
-    // operand of the k-th K step) while the loaders gather the first chunks
-    if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&bars[BAR_Q], TH * TD * 2);
-      for (int k = 0; k < TD / 16; ++k) tc::tma_load_2d(smem + OFF_Q + k * 4096, &qmap, 16 * k, row * TH, &bars[BAR_Q]);
+  // source row of item u of the list (selected entries, then the window);
+  // items past the list read the first window token (masked, P = 0)
+  auto item_src = [&](int u, const float **scp) -> const uint8_t * {
+    if (u < nsel) {
+      const int e = (SEL && a.idx) ? sel[u] : u;
+      const int64_t ent = (int64_t)b * a.entry_cap + e;
+      *scp = a.scales + ent;
+      return a.codes + ent * TD;
     }
-    // pull this CTA's gathered rows into L2 ahead of the loaders
-    const int u1 = min(c_end * CH, n_items);
-    for (int u = c_begin * CH + lane; u < u1; u += 32) {
-      const uint8_t *src;
-      if (u < nsel) src = a.codes + ((int64_t)b * a.entry_cap + (a.idx ? sel[u] : u)) * TD;
-      else src = a.wcodes + ((int64_t)b * a.win_cap + ((p0 + (u - nsel)) % a.win_cap)) * TD;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(TD) : "memory");
-    }
+    const int64_t p = p0 + (u < n_items ? u - nsel : 0);
+    const int64_t ent = (int64_t)b * a.win_cap + (p % a.win_cap);
+    *scp = a.wscales + ent;
+    return a.wcodes + ent * TD;
+  };
+  if (warp == 8 && lane == 0 && nloc > 0) {
+    // second half of Q: 16 boxes of 128 heads x 16 d (32-byte swizzle, the
+    // layout the MMA reads), box k = d 256 + 16 k
+    tc::mbar_arrive_expect_tx(&bars[BAR_Q], TH * (TD / 2) * 2);
+    for (int k = 0; k < TD / 32; ++k)
+      tc::tma_load_2d(smem + OFF_QH + k * 4096, &qmap, TD / 2 + 16 * k, row * TH, &bars[BAR_Q]);
   }
 
   if (warp < 4) {
     // ------------------------------------------------------------ loaders
+    // 4 threads per item row; warp w takes items 32 r + 8 w + (0..7) of
+    // each chunk, thread (i8, pq) the 16-byte groups pq + 4 k of the row:
+    // k < 4 lie in d < 256, k >= 4 in d >= 256.  Half A (d outside this
+    // CTA's output half) first, half B after; each half's loads for the next
+    // chunk are issued as soon as the previous half is stored.
     const int i8 = lane & 7, pq = lane >> 3;
+    const float qs = a.sm_scale * kLog2e;
+    const int u_end = min(c_end * CH, n_items);
+    const int ka = (1 - dh) * 4, kb = dh * 4;      // first k of half A / half B
+    uint4 ra[2][4], rb[2][4];
+    float sc[2];
+    auto load_half = [&](int lc, int k0, uint4 (&r)[2][4], bool with_scale) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int item = i * 32 + warp * 8 + i8;
+        const int u = (c_begin + lc) * CH + item;
+        const float *scp;
+        const uint8_t *src = item_src(u, &scp);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) r[i][k] = __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * (k0 + k));
+        if (with_scale) {
+          // consumed only when the half is stored (items past the list get 0
+          // there), so the load's latency stays hidden
+          sc[i] = __ldg(scp);
+        }
+      }
+      // dense lists: the entries of the chunk kPrefetchAhead ahead are
+      // contiguous rows; one bulk prefetch pulls them into L2
+      if (!SEL && with_scale && warp == 0 && lane == 0) {
+        const int f0 = (c_begin + lc + kPrefetchAhead) * CH;
+        const int f1 = min(min(f0 + CH, u_end), nsel);
+        if (f0 < f1)
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                       ::"l"(a.codes + ((int64_t)b * a.entry_cap + f0) * TD), "r"((f1 - f0) * TD) : "memory");
+      }
+    };
+    auto store_half = [&](unsigned char *kv, int k0, const uint4 (&r)[2][4]) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int item = i * 32 + warp * 8 + i8;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int p = pq + 4 * (k0 + k);
+          uint4 lo, hi;
+          e4m3x16_to_bf16x16(r[i][k], lo, hi);
+          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p)) = lo;
+          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p + 1)) = hi;
+        }
+      }
+    };
+    if (nloc > 0) {
+      load_half(0, ka, ra, false);
+      load_half(0, kb, rb, true);
+    }
     for (int lc = 0; lc < nloc; ++lc) {
-      const int buf = lc & 1;
-      const int item = warp * 8 + i8;
-      const int u = (c_begin + lc) * CH + item;
-      // Items past the list read a valid row (the first window token): their
-      // logits are masked and their P is zero, so the finite codes do not
-      // matter.  The loads are issued before waiting for the buffer.
-      const uint8_t *src;
-      const float *scp;
-      if (u < nsel) {
-        const int e = a.idx ? sel[u] : u;
-        const int64_t ent = (int64_t)b * a.entry_cap + e;
-        src = a.codes + ent * TD;
-        scp = a.scales + ent;
-      } else {
-        const int64_t p = p0 + (u < n_items ? u - nsel : 0);
-        const int64_t ent = (int64_t)b * a.win_cap + (p % a.win_cap);
-        src = a.wcodes + ent * TD;
-        scp = a.wscales + ent;
-      }
-      uint4 c[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) c[k] = __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * k);
-      const float sc_raw = __ldg(scp);
-      if (lc >= 2 && !wait_bar(&bars[BAR_KV_FREE + buf], ((lc - 2) >> 1) & 1, misc, a.status)) break;
-      const float sc = u < n_items ? sc_raw : 0.f;
-      unsigned char *kv = smem + OFF_KV + buf * KV_BYTES;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int p = pq + 4 * k;
-        uint4 lo, hi;
-        e4m3x16_to_bf16(c[k], lo, hi);
-        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p)) = lo;
-        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p + 1)) = hi;
-      }
-      if (pq == 0) iscale[buf * CH + item] = sc;
+      const int kslot = lc & 1;
+      unsigned char *kv = smem + OFF_KV + kslot * KV_BYTES;
+      // half A: free once QK(lc - 2) has read it
+      if (lc >= 2 && !wait_bar(&bars[BAR_FREE_A + kslot], ((lc - 2) >> 1) & 1, misc, a.status)) break;
+      store_half(kv, ka, ra);
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(&bars[BAR_KV_FULL + buf]);
+      tc::mbar_arrive(&bars[BAR_FULL_A + kslot]);
+      if (lc + 1 < nloc) load_half(lc + 1, ka, ra, false);
+      // half B and the item scales: free once PV(lc - 2) is done
+      if (lc >= 2 && !wait_bar(&bars[BAR_FREE_B + kslot], ((lc - 2) >> 1) & 1, misc, a.status)) break;
+      store_half(kv, kb, rb);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int item = i * 32 + warp * 8 + i8;
+        if (pq == 0) {
+          const float v = (c_begin + lc) * CH + item < n_items ? sc[i] : 0.f;
+          iscale[kslot * CH + item] = v;
+          lscale[kslot * CH + item] = v * qs;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars[BAR_FULL_B + kslot]);
+      if (lc + 1 < nloc) load_half(lc + 1, kb, rb, true);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
     const int quad = warp - 4;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const float qs = a.sm_scale * kLog2e;
-    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    if (nloc > 0) {
+      // first half of Q into TMEM: lane h, column 384 + j holds d = 2j, 2j + 1
+      const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + ((int64_t)row * TH + h) * TD);
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        uint32_t v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 x = __ldg(qrow + blk * 8 + k);
+          v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+        }
+        tc::tmem_st32(tbase + lane_off + TCOL_QL + blk * 32, v);
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars[BAR_QT]);
+    }
+    float m_used = -INFINITY, l = 0.f;
     for (int c = 0; c < nloc && ok; ++c) {
-      const int buf = c & 1;
-      // kv_full orders the loaders' scale writes before this thread's reads
+      const int buf = c & 1;          // S buffer and item tile
+      // full_b orders the loaders' scale writes before this thread's reads
       // one decision per warp: the TMEM accesses and votes below are warp-collective
-      if (!__all_sync(0xffffffffu, wait_bar(&bars[BAR_KV_FULL + buf], (c >> 1) & 1, misc, a.status) &&
+      if (!__all_sync(0xffffffffu, wait_bar(&bars[BAR_FULL_B + buf], (c >> 1) & 1, misc, a.status) &&
                                        wait_bar(&bars[BAR_S_FULL + buf], (c >> 1) & 1, misc, a.status))) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      uint32_t sr[32];
-      tc::tmem_ld32(tbase + lane_off + TCOL_S + buf * CH, sr);
-      tc::tmem_wait_ld();
       const int valid = min(CH, n_items - (c_begin + c) * CH);
-      float s[32];
+      const uint64_t *isc2 = reinterpret_cast<const uint64_t *>(iscale + buf * CH);
+      const uint64_t *lsc2 = reinterpret_cast<const uint64_t *>(lscale + buf * CH);
+      // logits in log2 units, as fp32 pairs: s = S * scale * softmax scale * log2(e)
+      uint64_t s2[CH / 2];
+      {
+        uint32_t sr[CH];
+#pragma unroll
+        for (int jb = 0; jb < CH / 32; ++jb)
+          tc::tmem_ld32(tbase + lane_off + TCOL_S + buf * CH + jb * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + jb * 32));
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < CH / 2; j += 2) {
+          const uint4 l4 = *reinterpret_cast<const uint4 *>(lsc2 + j);
+          s2[j] = mul2(pack2(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
+                       (uint64_t)l4.x | ((uint64_t)l4.y << 32));
+          s2[j + 1] = mul2(pack2(__uint_as_float(sr[2 * j + 2]), __uint_as_float(sr[2 * j + 3])),
+                           (uint64_t)l4.z | ((uint64_t)l4.w << 32));
+        }
+      }
+      if (valid < CH) {
+#pragma unroll
+        for (int j = 0; j < CH / 2; ++j) {
+          float x0, x1;
+          unpack2(s2[j], x0, x1);
+          s2[j] = pack2(2 * j < valid ? x0 : -INFINITY, 2 * j + 1 < valid ? x1 : -INFINITY);
+        }
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        s[j] = (j < valid) ? __uint_as_float(sr[j]) * iscale[buf * CH + j] * qs : -INFINITY;
-        mx = fmaxf(mx, s[j]);
+      for (int j = 0; j < CH / 2; ++j) {
+        float x0, x1;
+        unpack2(s2[j], x0, x1);
+        mx = max3(mx, x0, x1);
       }
       const bool need = mx > m_used + kRescaleLog2;
       if (c > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds earlier chunks: wait for the last PV, then rescale this warp's rows
+        // O holds earlier chunks: once PV(c - 1) is done, rescale this warp's rows
         if (!__all_sync(0xffffffffu, wait_bar(&bars[BAR_PV_DONE], (c - 1) & 1, misc, a.status))) { ok = false; break; }
         tc::fence_after_sync();
         const float f = need ? exp2f(m_used - mx) : 1.f;
@@ -327,21 +453,28 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
         l = (m_used == -INFINITY) ? 0.f : l * exp2f(m_used - mx);
         m_used = mx;
       }
-      uint32_t pw[16];
-      float lsum = 0.f;
+      // p = 2^(s - m); P = p * item scale, rounded to bf16
+      const uint64_t negm = pack2(-m_used, -m_used);
+      uint64_t lsum2 = pack2(0.f, 0.f);
+      uint32_t pw[CH / 2];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float pa = exp2f(s[j] - m_used), pb = exp2f(s[j + 1] - m_used);
-        lsum += pa + pb;
-        const __nv_bfloat162 v = __floats2bfloat162_rn(pa * iscale[buf * CH + j], pb * iscale[buf * CH + j + 1]);
-        pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+      for (int j = 0; j < CH / 2; ++j) {
+        float x0, x1;
+        unpack2(add2(s2[j], negm), x0, x1);
+        const uint64_t p2 = pack2(ex2(x0), ex2(x1));
+        lsum2 = add2(lsum2, p2);
+        float w0, w1;
+        unpack2(mul2(p2, isc2[j]), w0, w1);
+        const __nv_bfloat162 v = __floats2bfloat162_rn(w0, w1);
+        pw[j] = *reinterpret_cast<const uint32_t *>(&v);
       }
-      l += lsum;
-      unsigned char *P = smem + OFF_P + buf * P_BYTES;
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        *reinterpret_cast<uint4 *>(P + p_off(h, g)) = make_uint4(pw[4 * g], pw[4 * g + 1], pw[4 * g + 2], pw[4 * g + 3]);
-      tc::fence_proxy_async_smem();
+      float l0, l1;
+      unpack2(lsum2, l0, l1);
+      l += l0 + l1;
+      // P replaces the first 32 columns of its S buffer (row h, items
+      // 2j, 2j + 1 in column j), the A operand of the PV MMAs
+      tc::tmem_st32(tbase + lane_off + TCOL_S + buf * CH, pw);
+      tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars[BAR_P_FULL + buf]);
     }
@@ -396,47 +529,92 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   } else {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nloc > 0) {
-      const uint32_t idesc_qk = tc::idesc_bf16_f32(128, CH, 0, 0);
-      const uint32_t idesc_pv = tc::idesc_bf16_f32(128, DHALF, 0, 1);
-      auto issue_qk = [&](int c) {
+      constexpr uint32_t idesc_qk = tc::idesc_bf16_f32(128, CH, 0, 0);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, DHALF, 0, 1);
+      // Descriptors are built once; a K step only advances the start-address
+      // field (bits 0..13 hold address / 16, and every address in shared
+      // memory stays below 2^18, so the additions never carry out of it).
+      // QK B = items, K-major core matrices: LBO = step between d-groups, SBO = 8-row groups
+      const uint64_t bd_kv0 = tc::smem_desc(sbase + OFF_KV, GS, 128);
+      const uint64_t bd_kv1 = tc::smem_desc(sbase + OFF_KV + KV_BYTES, GS, 128);
+      // QK A (second half) = QH, K-major with 32-byte swizzle, one box per K step
+      const uint64_t ad_qh = tc::smem_desc_sw32(sbase + OFF_QH);
+      // PV A = P in TMEM (over its S buffer); B = the same item tile read
+      // MN-major (N = d): LBO = step between item groups (K), SBO = between d-groups (N)
+      const uint64_t bd_v0 = tc::smem_desc(sbase + OFF_KV + dh * (DHALF / 8) * GS, 128, GS);
+      const uint64_t bd_v1 = tc::smem_desc(sbase + OFF_KV + KV_BYTES + dh * (DHALF / 8) * GS, 128, GS);
+      // QK over one half of d: half 0 (d < 256) reads Q from TMEM, half 1
+      // from shared memory; accumulation starts with half A
+      auto issue_qk_half = [&](int c, int half, bool first) {
         const int buf = c & 1;
-        const uint32_t kvb = sbase + OFF_KV + buf * KV_BYTES;
-#pragma unroll 4
-        for (int k = 0; k < TD / 16; ++k) {
-          // A = Q, K-major with 32-byte swizzle (one TMA box per K step);
-          // B = items, K-major core matrices: LBO = step between d-groups, SBO = 8-row groups
-          const uint64_t ad = tc::smem_desc_sw32(sbase + OFF_Q + k * 4096);
-          const uint64_t bd = tc::smem_desc(kvb + k * 1024, 512, 128);
-          tc::mma_bf16_ss(tbase + TCOL_S + buf * CH, ad, bd, idesc_qk, k > 0);
-        }
-        tc::mma_commit(&bars[BAR_S_FULL + buf]);
-      };
-      bool ok = wait_bar(&bars[BAR_Q], 0, misc, a.status) && wait_bar(&bars[BAR_KV_FULL + 0], 0, misc, a.status);
-      if (ok) { tc::fence_after_sync(); issue_qk(0); }
-      if (ok && nloc > 1) {
-        ok = wait_bar(&bars[BAR_KV_FULL + 1], 0, misc, a.status);
-        if (ok) { tc::fence_after_sync(); issue_qk(1); }
-      }
-      for (int c = 0; c < nloc && ok; ++c) {
-        const int buf = c & 1;
-        if (!wait_bar(&bars[BAR_P_FULL + buf], (c >> 1) & 1, misc, a.status)) break;
-        tc::fence_after_sync();
-        const uint32_t pb = sbase + OFF_P + buf * P_BYTES;
-        const uint32_t vb = sbase + OFF_KV + buf * KV_BYTES + dh * (DHALF / 8) * 512;
+        const uint64_t bd = (buf ? bd_kv1 : bd_kv0) + (uint64_t)((half * (TD / 32) * 2 * GS) >> 4);
+        const uint32_t dt = tbase + TCOL_S + buf * CH;
+        if (half == 0) {
 #pragma unroll
-        for (int kk = 0; kk < CH / 16; ++kk) {
-          // A = P, K-major (K = items).  B = the same item tile read MN-major
-          // (N = d): LBO = step between item groups (K), SBO = between d-groups (N)
-          const uint64_t ad = tc::smem_desc(pb + kk * 4096, 2048, 128);
-          const uint64_t bd = tc::smem_desc(vb + kk * 256, 128, 512);
-          tc::mma_bf16_ss(tbase + TCOL_O, ad, bd, idesc_pv, (c > 0 || kk > 0));
+          for (int k = 0; k < TD / 32; ++k)
+            tc::mma_bf16_ts(dt, tbase + TCOL_QL + 8 * k, bd + (uint64_t)((k * 2 * GS) >> 4), idesc_qk, !first || k > 0);
+        } else {
+#pragma unroll
+          for (int k = 0; k < TD / 32; ++k)
+            tc::mma_bf16_ss(dt, ad_qh + (uint64_t)((k * 4096) >> 4), bd + (uint64_t)((k * 2 * GS) >> 4), idesc_qk,
+                            !first || k > 0);
         }
-        tc::mma_commit(&bars[BAR_KV_FREE + buf]);
+      };
+      auto issue_pv = [&](int c) {
+        const int buf = c & 1;
+        const uint64_t bd = buf ? bd_v1 : bd_v0;
+#pragma unroll
+        for (int kk = 0; kk < CH / 16; ++kk)
+          tc::mma_bf16_ts(tbase + TCOL_O, tbase + TCOL_S + buf * CH + 8 * kk, bd + (uint64_t)((kk * 256) >> 4), idesc_pv,
+                          (c > 0 || kk > 0));
+        tc::mma_commit(&bars[BAR_FREE_B + buf]);
         tc::mma_commit(&bars[BAR_PV_DONE]);
-        if (c + 2 < nloc) {
-          if (!wait_bar(&bars[BAR_KV_FULL + buf], ((c + 2) >> 1) & 1, misc, a.status)) break;
+      };
+      bool ok = wait_bar(&bars[BAR_Q], 0, misc, a.status) && wait_bar(&bars[BAR_QT], 0, misc, a.status);
+      // QK_A(c) (over half A) needs that half of tile c in place and S buffer
+      // c & 1 read (PV(c - 2) issued); QK_B(c) needs half B; PV(c) needs P(c).
+      // The first ready of PV, QK_B, QK_A goes next, so the tensor core works
+      // on one chunk while the loaders and the softmax warps handle others.
+      const int half_a = 1 - dh, half_b = dh;
+      int nqa = 0, nqb = 0, npv = 0;
+      const uint64_t t0 = globaltimer();
+      uint32_t spins = 0;
+      while (ok && npv < nloc) {
+        bool did = false;
+        const uint32_t pbar = BAR_P_FULL + (npv & 1);
+        const uint32_t ppar = (npv >> 1) & 1;
+        if (npv < nqb && tc::mbar_try_wait(&bars[pbar], ppar)) {
           tc::fence_after_sync();
-          issue_qk(c + 2);
+          issue_pv(npv);
+          ++npv;
+          did = true;
+        }
+        if (nqb < nqa && tc::mbar_try_wait(&bars[BAR_FULL_B + (nqb & 1)], (nqb >> 1) & 1)) {
+          tc::fence_after_sync();
+          issue_qk_half(nqb, half_b, false);
+          tc::mma_commit(&bars[BAR_S_FULL + (nqb & 1)]);
+          ++nqb;
+          did = true;
+        }
+        if (nqa < nloc && nqa < npv + 2 && tc::mbar_try_wait(&bars[BAR_FULL_A + (nqa & 1)], (nqa >> 1) & 1)) {
+          tc::fence_after_sync();
+          issue_qk_half(nqa, half_a, true);
+          tc::mma_commit(&bars[BAR_FREE_A + (nqa & 1)]);
+          ++nqa;
+          did = true;
+        }
+        if (did) {
+          spins = 0;
+          continue;
+        }
+        if ((++spins & 255u) == 0) {
+          if (*(volatile int *)&misc->abort) { ok = false; break; }
+          if (globaltimer() - t0 > kWaitNs * 4) {
+            misc->abort = 1;
+            raise_status(a.status, STATUS_TIMEOUT);
+            ok = false;
+            break;
+          }
         }
       }
       // drain: every MMA issued above has completed once FIN fires
@@ -553,7 +731,10 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
                        : nullptr;
   if (splits > 1 && !workspace) return fail(CSA_ERR_WORKSPACE, "attend: workspace required");
   a.status = status_word_device_ptr();
-  if (int rc = set_smem_once((const void *)attend_tc_kernel, (int)SMEM_BYTES, "attend_tc_kernel")) return rc;
+  // sparse instances keep room for the compacted selection
+  const void *kfn = dense ? (const void *)attend_tc_kernel<false> : (const void *)attend_tc_kernel<true>;
+  const uint32_t SMEM_BYTES = dense ? Lay<false>::SMEM_BYTES : Lay<true>::SMEM_BYTES;
+  if (int rc = set_smem_once(kfn, (int)SMEM_BYTES, "attend_tc_kernel")) return rc;
   const int64_t grid = rows * 2 * splits;
   if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "attend: too many rows");
   cudaLaunchConfig_t cfg = {};
@@ -573,7 +754,8 @@ int launch_attend_tc(const uint16_t *q, const uint8_t *codes, const float *scale
   if (!encode_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, TD, (uint64_t)(rows * TH), TD * 2, 16, TH,
                       CU_TENSOR_MAP_SWIZZLE_32B))
     return fail(CSA_ERR_INVALID, "attend: cannot map the queries for TMA (misaligned?)");
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_tc_kernel, qmap, a);
+  const cudaError_t e = dense ? cudaLaunchKernelEx(&cfg, attend_tc_kernel<false>, qmap, a)
+                              : cudaLaunchKernelEx(&cfg, attend_tc_kernel<true>, qmap, a);
   count_launches(1);
   if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "attend_tc_kernel launch: %s", cudaGetErrorString(e));
   return check_launch("attend_tc_kernel");

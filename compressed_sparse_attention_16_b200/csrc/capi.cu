@@ -119,10 +119,10 @@ bool encode_tmap_3d(CUtensorMap *map, CUtensorMapDataType type, const void *base
 }
 
 int set_smem_once(const void *kernel, int bytes, const char *name) {
-  // one slot per kernel instance that raises its limit: 27 in this library
-  // (the generic attention per D, the indexer paths per head count and
-  // indexer shape, the 128- and 64-head attention, the merge and the long
-  // pooling kernel), so 64 slots per device always suffice
+  // one slot per kernel instance that raises its limit (the generic
+  // attention per D, the indexer paths per head count and shape, the
+  // attention chunk shapes, the merges, the fused step and the long pooling
+  // kernel): fewer than 40 in this library, so 64 slots per device suffice
   constexpr int kSlots = 64;
   static std::mutex mu;
   static const void *done[64][kSlots] = {{nullptr}};

@@ -95,4 +95,30 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
+// Four E4M3 codes (low byte first) -> four bf16 (exact), as two bf16x2
+// words.  Byte s eeee mmm is placed at bf16 bits s 0000eeee mmm0000: for
+// e >= 1 that bf16 is 2^(e-127) (1 + m/8), for e = 0 the bf16 subnormal
+// (m/8) 2^-126, in both cases the code's value (2^(e-7) (1 + m/8), resp.
+// m 2^-9) times 2^-120; one bf16 multiply by 2^120 (bits 0x7B80) then
+// restores it exactly.  Integer placement and one multiply per pair replace
+// three conversion instructions.  The two NaN codes (0x7F, 0xFF), which
+// the library's quantiser never writes, come out as +-480.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  // 16-bit lanes [sign byte : code]: bytes 0, 1 (resp. 2, 3) of w with their
+  // sign bits replicated into the byte above
+  const uint32_t t0 = prmt(w, 0u, 0x9180u), t1 = prmt(w, 0u, 0xB3A2u);
+  const uint32_t y0 = ((t0 << 4) & 0x07F007F0u) | (t0 & 0x80008000u);
+  const uint32_t y1 = ((t1 << 4) & 0x07F007F0u) | (t1 & 0x80008000u);
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(y0), "r"(0x7B807B80u));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(y1), "r"(0x7B807B80u));
+}
+
+// 16 E4M3 codes -> 16 bf16 (exact), as two 16-byte words
+__device__ __forceinline__ void e4m3x16_to_bf16x16(const uint4 &c, uint4 &lo, uint4 &hi) {
+  e4m3x4_to_bf16x4(c.x, lo.x, lo.y);
+  e4m3x4_to_bf16x4(c.y, lo.z, lo.w);
+  e4m3x4_to_bf16x4(c.z, hi.x, hi.y);
+  e4m3x4_to_bf16x4(c.w, hi.z, hi.w);
+}
+
 }  // namespace csa

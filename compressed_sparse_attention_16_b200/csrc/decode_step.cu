@@ -405,21 +405,6 @@ __device__ __forceinline__ uint32_t quant4(const float (&C)[4], float s) {
 __device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 2048 + (i >> 3) * 128 + (i & 7) * 16; }
 __device__ __forceinline__ uint32_t p_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
 
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 &c, uint4 &lo, uint4 &hi) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 a = e4m3x2_to_float2((uint16_t)(w[k] & 0xFFFF));
-    const float2 b = e4m3x2_to_float2((uint16_t)(w[k] >> 16));
-    const __nv_bfloat162 ab = __float22bfloat162_rn(a);
-    const __nv_bfloat162 bb = __float22bfloat162_rn(b);
-    o[2 * k] = *reinterpret_cast<const uint32_t *>(&ab);
-    o[2 * k + 1] = *reinterpret_cast<const uint32_t *>(&bb);
-  }
-  lo = make_uint4(o[0], o[1], o[2], o[3]);
-  hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
 
 __device__ __forceinline__ uint4 ldcg16(const void *p) { return __ldcg(reinterpret_cast<const uint4 *>(p)); }
 
@@ -1019,7 +1004,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         for (int k = 0; k < 8; ++k) {
           const int pc = pq + 4 * k;
           uint4 lo, hi;
-          e4m3x16_to_bf16(cv[r][k], lo, hi);
+          e4m3x16_to_bf16x16(cv[r][k], lo, hi);
           *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * pc)) = lo;
           *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * pc + 1)) = hi;
         }

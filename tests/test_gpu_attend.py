@@ -9,6 +9,7 @@ import compressed_sparse_attention_16_b200 as csa
 import synth
 from compressed_sparse_attention_16_b200 import Dims
 from oracle import csa as ocsa
+from oracle.formats import e4m3_decode
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -172,3 +173,38 @@ def test_wide_dynamic_range(H, qexp, sexp):
     out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
     ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % win_cap], q_pos, W, scale=D ** -0.5)
     parity.check_attention(out, lse, ro, rl)
+
+
+def _all_codes_row(D):
+    """D E4M3 codes: column d holds byte d mod 256, except the two NaN codes
+    (0x7F, 0xFF), which the library's quantiser never writes, set to 0.  Each
+    256-column half of D = 512 holds every finite code, subnormals included."""
+    c = (np.arange(D) % 256).astype(np.uint8)
+    c[(c == 0x7F) | (c == 0xFF)] = 0
+    return c
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_every_e4m3_code_decodes_exactly(dense):
+    """Every attended item holds the same codes (every finite E4M3 byte, in
+    both halves of D) with scale 1, so all logits are equal, every weight is
+    exactly 1 / n and the output row is the decoded codes: each code's bf16
+    image must come out exactly, the 7 subnormal magnitudes and the zeros
+    included.  (The fused decode step shares the same
+    conversion.)  A per-row tolerance could not see a wrong subnormal."""
+    B, Tq, H, D, m, N, K, W = 2, 3, 128, 512, 4, 700, 512, 128
+    row = _all_codes_row(D)
+    codes = torch.from_numpy(np.broadcast_to(row, (B, N, D)).copy())
+    wcodes = torch.from_numpy(np.broadcast_to(row, (B, W, D)).copy())
+    scales = torch.ones((B, N), dtype=torch.float32)
+    wscales = torch.ones((B, W), dtype=torch.float32)
+    q = synth.queries(B, Tq, H, D, 512 ** -0.5, 5)
+    q_pos = np.array([[m * N - 1, 1000, 3]] * B, dtype=np.int32)
+    rng = np.random.default_rng(7)
+    idx = None if dense else _random_selection(rng, q_pos, m, N, K)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=W)
+    out, _ = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+    want = torch.from_numpy(e4m3_decode(row)).to(torch.bfloat16)
+    got = out.cpu()
+    assert torch.equal(got, want.expand_as(got)), (
+        f"{int((got != want.expand_as(got)).sum())} outputs differ from the decoded codes")
