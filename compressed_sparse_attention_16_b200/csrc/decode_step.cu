@@ -36,11 +36,12 @@
 //   B   attend: every CTA becomes one attention unit (sequence, quarter of
 //       D, item split) and runs the tensor-core MQA over its chunks of the
 //       sequence's item list (selected entries, then window tokens).  Q lives
-//       in TMEM as the A operand of S = Q K^T (M = 128 heads, N = 32 items,
+//       in TMEM as the A operand of S = Q K^T (M = 128 heads, N = 128 items,
 //       K = 512), so the tensor core streams only the item tile from shared
-//       memory; E4M3 rows are converted exactly to bf16; the softmax (one head
-//       per thread, lazy rescaling) writes P = p * item scale straight into
-//       TMEM as the A operand of O += P V (N = 128, the unit's quarter of D).
+//       memory; E4M3 rows are converted exactly to bf16; the softmax (two
+//       threads per head, 64 items each, one pass over S, lazy rescaling)
+//       writes P = p * item scale straight into TMEM over S, the A operand
+//       of O += P V (N = 128, the unit's quarter of D).
 //       Item splits write unnormalised partials and count themselves done
 //       per (sequence, quarter); each unit then merges its share of the heads.
 //
@@ -90,9 +91,7 @@ constexpr uint32_t A_END = A_QI + 256;
 constexpr uint32_t B_Q = 0;
 constexpr uint32_t B_KV = 0;
 constexpr uint32_t KV_BYTES = CH * TD * 2;                      // 128 KiB
-constexpr uint32_t B_P = B_KV + KV_BYTES;                       // P [128 heads][128 items] bf16
-constexpr uint32_t P_BYTES = TH * CH * 2;                       // 32 KiB
-constexpr uint32_t B_SEL = B_P + P_BYTES;                       // int32 [kMaxSelLocal]
+constexpr uint32_t B_SEL = B_KV + KV_BYTES;                     // int32 [kMaxSelLocal]
 constexpr uint32_t B_SCALE = B_SEL + kMaxSelLocal * 4;          // fp32 [128] item scales
 constexpr uint32_t B_MX = B_SCALE + CH * 4;                     // fp32 [2][128] per-half maxima / sums
 constexpr uint32_t B_END = B_MX + 2 * TH * 4;
@@ -399,11 +398,9 @@ __device__ __forceinline__ uint32_t quant4(const float (&C)[4], float s) {
 // ---------------------------------------------------------------------------
 // attention helpers
 // ---------------------------------------------------------------------------
-// Core-matrix layouts (8 rows x 16 B): the item tile KV [128 items][512 d]
-// with g = d / 8, g-stride 2 KiB and item-group stride 128 B; P [128 heads]
-// [128 items] with g = item / 8, g-stride 2 KiB and head-group stride 128 B.
+// Core-matrix layout (8 rows x 16 B) of the item tile KV [128 items][512 d]:
+// g = d / 8, g-stride 2 KiB, item-group stride 128 B.
 __device__ __forceinline__ uint32_t kv_off(int i, int g) { return g * 2048 + (i >> 3) * 128 + (i & 7) * 16; }
-__device__ __forceinline__ uint32_t p_off(int h, int g) { return g * 2048 + (h >> 3) * 128 + (h & 7) * 16; }
 
 
 __device__ __forceinline__ uint4 ldcg16(const void *p) { return __ldcg(reinterpret_cast<const uint4 *>(p)); }
@@ -1017,17 +1014,20 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       tc::fence_after_sync();
       const int valid = min(CH, n_items - (c_begin + c) * CH);
       const int i_lo = half * (CH / 2);
-      float pmx = -INFINITY;
-#pragma unroll 1
-      for (int jb = 0; jb < CH / 64; ++jb) {
-        uint32_t sr[32];
-        tc::tmem_ld32(tbase + lane_off + TCOL_S + i_lo + jb * 32, sr);
-        tc::tmem_wait_ld();
+      // one pass over this half's 64 scores: all of them into registers
+      // (every TMEM read of S is done before the half's P overwrites part of S)
+      uint32_t sr[CH / 2];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = i_lo + jb * 32 + j;
-          if (i < valid) pmx = fmaxf(pmx, __uint_as_float(sr[j]) * iscale[i] * qs);
-        }
+      for (int jb = 0; jb < CH / 64; ++jb)
+        tc::tmem_ld32(tbase + lane_off + TCOL_S + i_lo + jb * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + jb * 32));
+      tc::tmem_wait_ld();
+      float sv[CH / 2];
+      float pmx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < CH / 2; ++j) {
+        const int i = i_lo + j;
+        sv[j] = i < valid ? __uint_as_float(sr[j]) * iscale[i] * qs : -INFINITY;
+        pmx = fmaxf(pmx, sv[j]);
       }
       // the two halves agree on the chunk maximum through shared memory
       mxx[half * TH + h] = pmx;
@@ -1056,33 +1056,22 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         l_sum = (m_used == -INFINITY) ? 0.f : l_sum * ex2(m_used - mx);
         m_used = mx;
       }
-      // P = p * item scale (bf16) for this half's items, in the core-matrix
-      // layout of the PV A operand
-      unsigned char *P = smem + B_P;
+      // P = p * item scale (bf16) for this half's items into TMEM over the
+      // first 64 columns of S (row h, items 2j, 2j + 1 in column j): half h
+      // writes columns 32 half .. 32 half + 31, the A operand of the PV MMAs
       float lsum = 0.f;
-#pragma unroll 1
-      for (int jb = 0; jb < CH / 64; ++jb) {
-        uint32_t sr[32];
-        tc::tmem_ld32(tbase + lane_off + TCOL_S + i_lo + jb * 32, sr);
-        tc::tmem_wait_ld();
-        uint32_t pw[16];
+      uint32_t pw[32];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const int i0 = i_lo + jb * 32 + j;
-          const float sa = i0 < valid ? __uint_as_float(sr[j]) * iscale[i0] * qs : -INFINITY;
-          const float sb = i0 + 1 < valid ? __uint_as_float(sr[j + 1]) * iscale[i0 + 1] * qs : -INFINITY;
-          const float pa = ex2(sa - m_used), pb = ex2(sb - m_used);
-          lsum += pa + pb;
-          const __nv_bfloat162 v = __floats2bfloat162_rn(pa * iscale[i0], pb * iscale[i0 + 1]);
-          pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
-        }
-#pragma unroll
-        for (int gg = 0; gg < 4; ++gg)
-          *reinterpret_cast<uint4 *>(P + p_off(h, (i_lo + jb * 32) / 8 + gg)) =
-              make_uint4(pw[4 * gg], pw[4 * gg + 1], pw[4 * gg + 2], pw[4 * gg + 3]);
+      for (int j = 0; j < CH / 2; j += 2) {
+        const int i0 = i_lo + j;
+        const float pa = ex2(sv[j] - m_used), pb = ex2(sv[j + 1] - m_used);
+        lsum += pa + pb;
+        const __nv_bfloat162 v = __floats2bfloat162_rn(pa * iscale[i0], pb * iscale[i0 + 1]);
+        pw[j >> 1] = *reinterpret_cast<const uint32_t *>(&v);
       }
+      tc::tmem_st32(tbase + lane_off + TCOL_S + half * 32, pw);
+      tc::tmem_wait_st();
       l_sum += lsum;
-      tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       tc::mbar_arrive(&bar[BAR_P_FULL]);
     }
@@ -1164,13 +1153,14 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
         tc::mma_commit(&bar[BAR_S_FULL]);
         if (!bwait(&bar[BAR_P_FULL], c & 1, misc, a.status)) break;
         tc::fence_after_sync();
-        // O += P V: A = P (K-major, K = items), B = the item tile read MN-major
-        // for this quarter of D (LBO = item-group step, SBO = d-group step)
+        // O += P V: A = P in TMEM over S (8 columns per 16 items), B = the
+        // item tile read MN-major for this quarter of D (LBO = item-group
+        // step, SBO = d-group step)
         const uint32_t vb = sbase + B_KV + qd * (DQ / 8) * 2048;
 #pragma unroll
         for (int kk = 0; kk < CH / 16; ++kk)
-          tc::mma_bf16_ss(tbase + TCOL_O, tc::smem_desc(sbase + B_P + kk * 4096, 2048, 128),
-                          tc::smem_desc(vb + kk * 256, 128, 2048), idesc_pv, (c > 0 || kk > 0));
+          tc::mma_bf16_ts(tbase + TCOL_O, tbase + TCOL_S + 8 * kk, tc::smem_desc(vb + kk * 256, 128, 2048), idesc_pv,
+                          (c > 0 || kk > 0));
         tc::mma_commit(&bar[BAR_KV_FREE]);
         tc::mma_commit(&bar[BAR_PV_DONE]);
       }
