@@ -190,6 +190,65 @@ struct Args {
   unsigned *status;
 };
 
+// Combine the S <= JMAX split partials of `nh` (<= NH) heads h0, h0 + 8, ...
+// of one (row, half) into the bf16 output (and the log-sum-exp):
+//   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
+// Lane l handles d = 8 l .. 8 l + 7 of the half; all loads are issued first.
+template <int JMAX, int NH>
+__device__ __forceinline__ void merge_heads(const Args &a, int64_t slot0, int S, int h0, int nh, int row, int dh,
+                                            int lane) {
+  float2 ml[NH];
+  float4 v0[NH][JMAX], v1[NH][JMAX];
+#pragma unroll
+  for (int n = 0; n < NH; ++n) {
+    const int h = h0 + 8 * n;
+    const bool live = n < nh;
+    ml[n] = (live && lane < S) ? __ldcg(a.ws_ml + (slot0 + lane) * TH + h) : make_float2(-INFINITY, 0.f);
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      v0[n][j] = v1[n][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (live && j < S) {
+        // d = 8 lane .. 8 lane + 7: block lane / 4, offset 8 (lane % 4)
+        const float4 *src = reinterpret_cast<const float4 *>(
+            a.ws_o + (slot0 + j) * TH * DHALF + ((int64_t)(lane >> 2) * TH + h) * 32 + (lane & 3) * 8);
+        v0[n][j] = __ldcg(src);
+        v1[n][j] = __ldcg(src + 1);
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NH; ++n) {
+    if (n >= nh) break;
+    const int h = h0 + 8 * n;
+    float M = ml[n].x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wgt = (ml[n].y > 0.f) ? exp2f(ml[n].x - M) : 0.f;
+    float L = wgt * ml[n].y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+#pragma unroll
+    for (int j = 0; j < JMAX; ++j) {
+      const float wj = __shfl_sync(0xffffffffu, wgt, j);
+      acc[0] += wj * v0[n][j].x; acc[1] += wj * v0[n][j].y; acc[2] += wj * v0[n][j].z; acc[3] += wj * v0[n][j].w;
+      acc[4] += wj * v1[n][j].x; acc[5] += wj * v1[n][j].y; acc[6] += wj * v1[n][j].z; acc[7] += wj * v1[n][j].w;
+    }
+    const float inv = 1.f / L;
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      const __nv_bfloat162 v = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
+      w[k >> 1] = *reinterpret_cast<const uint32_t *>(&v);
+    }
+    const int64_t orow = (int64_t)row * TH + h;
+    *reinterpret_cast<uint4 *>(a.out + orow * TD + dh * DHALF + lane * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (a.lse && dh == 0 && lane == 0) a.lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
+  }
+}
+
 template <bool SEL>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_constant__ CUtensorMap qmap,
                                                                 const Args a) {
@@ -510,19 +569,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       // thread writes whole 128-byte lines
       const int64_t slot = (int64_t)pair * a.splits + split;
       float *dstb = a.ws_o + slot * TH * DHALF;
+      // two 32-column blocks per round: both TMEM loads in flight together
 #pragma unroll 1
-      for (int blk = 0; blk < DHALF / 32; ++blk) {
-        uint32_t o[32];
+      for (int blk = 0; blk < DHALF / 32; blk += 2) {
+        uint32_t o[2][32];
         if (have) {
-          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o);
+          tc::tmem_ld32(tbase + lane_off + TCOL_O + blk * 32, o[0]);
+          tc::tmem_ld32(tbase + lane_off + TCOL_O + (blk + 1) * 32, o[1]);
           tc::tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = 0u;
+          for (int j = 0; j < 32; ++j) o[0][j] = o[1][j] = 0u;
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(dstb + ((int64_t)blk * TH + h) * 32);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        for (int u = 0; u < 2; ++u) {
+          uint4 *dst = reinterpret_cast<uint4 *>(dstb + ((int64_t)(blk + u) * TH + h) * 32);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) dst[k] = make_uint4(o[u][4 * k], o[u][4 * k + 1], o[u][4 * k + 2], o[u][4 * k + 3]);
+        }
       }
       a.ws_ml[slot * TH + h] = have ? make_float2(m_used, l) : make_float2(-INFINITY, 0.f);
     }
@@ -636,48 +700,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     const int hper = TH / S;
     if (warp < 8) {
       const int64_t slot0 = (int64_t)pair * S;
-      for (int hl = warp; hl < hper; hl += 8) {
-        const int h = split * hper + hl;
-        const float2 ml = lane < S ? __ldcg(a.ws_ml + (slot0 + lane) * TH + h) : make_float2(-INFINITY, 0.f);
-        // every source's row in flight before any use
-        float4 v0[8], v1[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v0[j] = v1[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < S) {
-            // d = 8 lane .. 8 lane + 7: block lane / 4, offset 8 (lane % 4)
-            const float4 *src = reinterpret_cast<const float4 *>(
-                a.ws_o + (slot0 + j) * TH * DHALF + ((int64_t)(lane >> 2) * TH + h) * 32 + (lane & 3) * 8);
-            v0[j] = __ldcg(src);
-            v1[j] = __ldcg(src + 1);
-          }
-        }
-        float M = ml.x;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        const float wgt = (ml.y > 0.f) ? exp2f(ml.x - M) : 0.f;
-        float L = wgt * ml.y;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float wj = __shfl_sync(0xffffffffu, wgt, j);
-          acc[0] += wj * v0[j].x; acc[1] += wj * v0[j].y; acc[2] += wj * v0[j].z; acc[3] += wj * v0[j].w;
-          acc[4] += wj * v1[j].x; acc[5] += wj * v1[j].y; acc[6] += wj * v1[j].z; acc[7] += wj * v1[j].w;
-        }
-        const float inv = 1.f / L;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 8; k += 2) {
-          const __nv_bfloat162 v = __floats2bfloat162_rn(acc[k] * inv, acc[k + 1] * inv);
-          w[k >> 1] = *reinterpret_cast<const uint32_t *>(&v);
-        }
-        const int64_t orow = (int64_t)row * TH + h;
-        *reinterpret_cast<uint4 *>(a.out + orow * TD + dh * DHALF + lane * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        if (a.lse && dh == 0 && lane == 0) a.lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
+      // S <= 4: two heads per round, so both heads' partials are in flight together
+      if (S <= 4) {
+        for (int hl = warp; hl < hper; hl += 16)
+          merge_heads<4, 2>(a, slot0, S, split * hper + hl, hl + 8 < hper ? 2 : 1, row, dh, lane);
+      } else {
+        for (int hl = warp; hl < hper; hl += 8) merge_heads<8, 1>(a, slot0, S, split * hper + hl, 1, row, dh, lane);
       }
     }
   }
