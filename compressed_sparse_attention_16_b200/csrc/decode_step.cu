@@ -890,8 +890,14 @@ decode_step_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_consta
       for (uint32_t j = lane; j < nc; j += 32) r += ck[j] > key ? 1u : 0u;
       r = __reduce_add_sync(0xffffffffu, r);
       if (lane == 0 && r < (uint32_t)cnt) {
-        oi[r] = (int32_t)(0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu));
+        const uint32_t e = 0xFFFFFFFFu - (uint32_t)(key & 0xFFFFFFFFu);
+        oi[r] = (int32_t)e;
         if (os) os[r] = (float)(uint32_t)(key >> 32) * (1.f / 64.f);
+        // the attention gathers this row next (the candidates of a tie-flooded
+        // threshold bin were not prefetched when they were listed)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.codes + ((int64_t)rowA * a.entry_cap + e) * TD),
+                     "r"(TD)
+                     : "memory");
       }
     }
     if (part == 0) {
