@@ -216,6 +216,121 @@ compress_tokens_kernel(const float *__restrict__ x, const float *__restrict__ z,
   }
 }
 
+// Large blocks on many SMs (m >= 16, D a multiple of 64): the channels of
+// one entry are split over a thread-block cluster of D / 64 CTAs (the
+// softmax is per channel, so the CTAs pool independently); in each CTA 16
+// token groups of 16 threads run the online softmax over tokens g, g + 16,
+// ... for 4 channels each, and the 16 partial states are merged per channel
+// in shared memory.  Only the entry's amax couples the channels: each CTA
+// publishes its 64-channel amax and reads the others' through distributed
+// shared memory, so every CTA derives the same scale and quantises its own
+// channels.
+constexpr int kClChannels = 64;                   // channels per CTA
+constexpr int kClGroups = 16;                     // token groups per CTA
+constexpr int kClThreads = kClGroups * (kClChannels / 4);
+
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float cl_load_f32(const float *p, uint32_t rank) {
+  uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p)), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(r) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kClThreads)
+compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_per_seq, int D, int m,
+                        int64_t x_bstride, uint8_t *__restrict__ codes, float *__restrict__ scales,
+                        int64_t dst_first, int64_t dst_bstride, int ring_cap, float *__restrict__ pooled) {
+  __shared__ float part[3][kClGroups][kClChannels];   // max, normaliser, weighted sum
+  __shared__ float cpool[kClChannels];
+  __shared__ float wmax[kClChannels / 32];
+  __shared__ float amax_cta;
+  const int CG = D / kClChannels;                     // CTAs per entry (= cluster size)
+  const int rank = (int)(blockIdx.x % CG);
+  const int64_t e = blockIdx.x / CG;
+  const int64_t b = e / n_per_seq, i = e - b * n_per_seq;
+  // with a ring only the call's last ring_cap blocks survive (the whole
+  // cluster leaves together, before its barriers)
+  if (ring_cap > 0 && i + ring_cap < n_per_seq) return;
+  const int L = kClChannels / 4;
+  const int g = threadIdx.x / L, lane = threadIdx.x - g * L;
+  const int64_t col = (int64_t)rank * L + lane;       // float4 column of the row
+  const float4 *xp = reinterpret_cast<const float4 *>(x + b * x_bstride + i * (int64_t)m * D) + col;
+  const float4 *zp = reinterpret_cast<const float4 *>(z + b * x_bstride + i * (int64_t)m * D) + col;
+  const int64_t rs = D / 4;                           // float4 per token row
+  OnlineSoftmax4 sm;
+  sm.init();
+  // up to 8 tokens per thread in flight together (one HBM round trip for m <= 128)
+  constexpr int kClUnroll = 8;
+  int j = g;
+  for (; j + (kClUnroll - 1) * kClGroups < m; j += kClUnroll * kClGroups) {
+    float4 xv[kClUnroll], zv[kClUnroll];
+#pragma unroll
+    for (int u = 0; u < kClUnroll; ++u) {
+      xv[u] = __ldg(xp + (int64_t)(j + u * kClGroups) * rs);
+      zv[u] = __ldg(zp + (int64_t)(j + u * kClGroups) * rs);
+    }
+#pragma unroll
+    for (int u = 0; u < kClUnroll; ++u) sm.push(xv[u], zv[u]);
+  }
+  for (; j < m; j += kClGroups) sm.push(__ldg(xp + (int64_t)j * rs), __ldg(zp + (int64_t)j * rs));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    part[0][g][4 * lane + c] = sm.mx[c];
+    part[1][g][4 * lane + c] = sm.l[c];
+    part[2][g][4 * lane + c] = sm.acc[c];
+  }
+  __syncthreads();
+  if (threadIdx.x < kClChannels) {
+    const int ch = threadIdx.x;
+    float M = -INFINITY;
+    for (int k = 0; k < kClGroups; ++k) M = fmaxf(M, part[0][k][ch]);
+    float l = 0.f, acc = 0.f;
+    for (int k = 0; k < kClGroups; ++k) {
+      const float mk = part[0][k][ch];
+      if (mk == -INFINITY) continue;                  // a group that saw no token
+      const float f = expf(mk - M);
+      l = fmaf(part[1][k][ch], f, l);
+      acc = fmaf(part[2][k][ch], f, acc);
+    }
+    const float C = __fdiv_rn(acc, l);
+    cpool[ch] = C;
+    float a = fabsf(C);
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((ch & 31) == 0) wmax[ch >> 5] = a;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) amax_cta = fmaxf(wmax[0], wmax[1]);
+  // every CTA's amax visible to the cluster
+  cl_sync();
+  float a = 0.f;
+  for (int r = 0; r < CG; ++r) a = fmaxf(a, cl_load_f32(&amax_cta, (uint32_t)r));
+  float s = __fdiv_rn(a, 448.f);
+  if (!(s > 0.f)) s = 1.f;
+  int64_t slot = dst_first + i;
+  if (ring_cap > 0) slot %= ring_cap;
+  const int64_t ent = b * dst_bstride + slot;
+  if (threadIdx.x < L) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t q = __nv_cvt_float_to_fp8(__fdiv_rn(cpool[4 * threadIdx.x + c], s), __NV_SATFINITE, __NV_E4M3);
+      word |= q << (8 * c);
+    }
+    reinterpret_cast<uint32_t *>(codes + ent * D)[rank * L + threadIdx.x] = word;
+    if (pooled)
+      reinterpret_cast<float4 *>(pooled + (b * n_per_seq + i) * (int64_t)D)[rank * L + threadIdx.x] =
+          make_float4(cpool[4 * threadIdx.x], cpool[4 * threadIdx.x + 1], cpool[4 * threadIdx.x + 2],
+                      cpool[4 * threadIdx.x + 3]);
+  }
+  if (rank == 0 && threadIdx.x == 0) scales[ent] = s;
+  // no CTA leaves while another may still read its amax
+  cl_sync();
+}
+
 // Entries and window in one pass: each group of D/4 threads pools one block
 // of m tokens (m = 2, 4 or 8) into an entry exactly as compress_kernel does,
 // and also quantises each of the block's m tokens on its own as a window
@@ -378,6 +493,29 @@ int launch_compress(const float *x, const float *z, int B, int T, int D, int m, 
   const int64_t total = (int64_t)B * n;
   if (total == 0) return CSA_OK;
   const int L = D / 4;
+  if (m >= 16 && D % kClChannels == 0 && D / kClChannels <= 8) {
+    // channel-split clusters: D / 64 CTAs per entry
+    const int CG = D / kClChannels;
+    const int64_t grid = total * CG;
+    if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: too many entries");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, compress_cluster_kernel, x, z, n, D, m, x_bstride, codes, scales,
+                                             dst_first, dst_bstride, ring_cap, pooled);
+    count_launches(1);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "compress_cluster_kernel launch: %s", cudaGetErrorString(e));
+    return check_launch("compress_cluster_kernel");
+  }
   if (m >= 16 && L <= 512) {
     int G = 1024 / L;
     while (G > 1 && G * 8 > m) G >>= 1;                 // at least 8 tokens per group
