@@ -224,10 +224,14 @@ compress_tokens_kernel(const float *__restrict__ x, const float *__restrict__ z,
 // in shared memory.  Only the entry's amax couples the channels: each CTA
 // publishes its 64-channel amax and reads the others' through distributed
 // shared memory, so every CTA derives the same scale and quantises its own
-// channels.
+// channels.  With window outputs (wcodes, m <= 128 and a multiple of 16:
+// every token is in registers), each of the block's tokens is also
+// quantised on its own exactly as the one-token rule does (C = x, s = amax /
+// 448, the token's amax shared the same way), so the tokens are read once.
 constexpr int kClChannels = 64;                   // channels per CTA
 constexpr int kClGroups = 16;                     // token groups per CTA
 constexpr int kClThreads = kClGroups * (kClChannels / 4);
+constexpr int kClUnroll = 8;                      // tokens per thread in one batch; window fusion needs m = 128
 
 __device__ __forceinline__ void cl_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -243,9 +247,13 @@ __device__ __forceinline__ float cl_load_f32(const float *p, uint32_t rank) {
 __global__ void __launch_bounds__(kClThreads)
 compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z, int n_per_seq, int D, int m,
                         int64_t x_bstride, uint8_t *__restrict__ codes, float *__restrict__ scales,
-                        int64_t dst_first, int64_t dst_bstride, int ring_cap, float *__restrict__ pooled) {
+                        int64_t dst_first, int64_t dst_bstride, int ring_cap, float *__restrict__ pooled,
+                        int T, uint8_t *__restrict__ wcodes, float *__restrict__ wscales, int64_t w_first,
+                        int64_t w_bstride, int w_ring) {
   __shared__ float part[3][kClGroups][kClChannels];   // max, normaliser, weighted sum
   __shared__ float cpool[kClChannels];
+  __shared__ float tok_amax[kClGroups * 8];           // window: this CTA's 64-channel amax per token
+  __shared__ float tok_scale[kClGroups * 8];
   __shared__ float wmax[kClChannels / 32];
   __shared__ float amax_cta;
   const int CG = D / kClChannels;                     // CTAs per entry (= cluster size)
@@ -254,7 +262,9 @@ compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z
   const int64_t b = e / n_per_seq, i = e - b * n_per_seq;
   // with a ring only the call's last ring_cap blocks survive (the whole
   // cluster leaves together, before its barriers)
-  if (ring_cap > 0 && i + ring_cap < n_per_seq) return;
+  const bool win = wcodes != nullptr;                 // the host fuses only when m <= 128, m % 16 == 0
+  if (!win && ring_cap > 0 && i + ring_cap < n_per_seq) return;
+  const bool entry_live = !(ring_cap > 0 && i + ring_cap < n_per_seq);
   const int L = kClChannels / 4;
   const int g = threadIdx.x / L, lane = threadIdx.x - g * L;
   const int64_t col = (int64_t)rank * L + lane;       // float4 column of the row
@@ -264,7 +274,7 @@ compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z
   OnlineSoftmax4 sm;
   sm.init();
   // up to 8 tokens per thread in flight together (one HBM round trip for m <= 128)
-  constexpr int kClUnroll = 8;
+  float4 keep[kClUnroll];
   int j = g;
   for (; j + (kClUnroll - 1) * kClGroups < m; j += kClUnroll * kClGroups) {
     float4 xv[kClUnroll], zv[kClUnroll];
@@ -275,6 +285,18 @@ compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z
     }
 #pragma unroll
     for (int u = 0; u < kClUnroll; ++u) sm.push(xv[u], zv[u]);
+    if (win) {
+      // window (m = 128: this is the thread's only batch): each token's amax
+      // over this CTA's channels (the 16 lanes of a token group are one half
+      // of a warp); the tokens stay in registers for their codes below
+#pragma unroll
+      for (int u = 0; u < kClUnroll; ++u) {
+        float t = fmaxf(fmaxf(fabsf(xv[u].x), fabsf(xv[u].y)), fmaxf(fabsf(xv[u].z), fabsf(xv[u].w)));
+        for (int o = 8; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+        if (lane == 0) tok_amax[g + u * kClGroups] = t;
+        keep[u] = xv[u];
+      }
+    }
   }
   for (; j < m; j += kClGroups) sm.push(__ldg(xp + (int64_t)j * rs), __ldg(zp + (int64_t)j * rs));
 #pragma unroll
@@ -313,7 +335,7 @@ compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z
   int64_t slot = dst_first + i;
   if (ring_cap > 0) slot %= ring_cap;
   const int64_t ent = b * dst_bstride + slot;
-  if (threadIdx.x < L) {
+  if (threadIdx.x < L && entry_live) {
     uint32_t word = 0;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -326,8 +348,36 @@ compress_cluster_kernel(const float *__restrict__ x, const float *__restrict__ z
           make_float4(cpool[4 * threadIdx.x], cpool[4 * threadIdx.x + 1], cpool[4 * threadIdx.x + 2],
                       cpool[4 * threadIdx.x + 3]);
   }
-  if (rank == 0 && threadIdx.x == 0) scales[ent] = s;
-  // no CTA leaves while another may still read its amax
+  if (rank == 0 && threadIdx.x == 0 && entry_live) scales[ent] = s;
+  if (win) {
+    // each token's scale from the cluster's per-token amaxima, then its codes
+    if (threadIdx.x < m) {
+      float ta = 0.f;
+      for (int r = 0; r < CG; ++r) ta = fmaxf(ta, cl_load_f32(&tok_amax[threadIdx.x], (uint32_t)r));
+      float ts = __fdiv_rn(ta, 448.f);
+      if (!(ts > 0.f)) ts = 1.f;
+      tok_scale[threadIdx.x] = ts;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kClUnroll; ++u) {
+      const int jt = g + u * kClGroups;               // token within the block
+      const int64_t t = i * (int64_t)m + jt;          // token within the call
+      if (w_ring > 0 && t + w_ring < T) continue;     // overwritten later in this call
+      int64_t wslot = w_first + t;
+      if (w_ring > 0) wslot %= w_ring;
+      const int64_t went = b * w_bstride + wslot;
+      const float ts = tok_scale[jt];
+      const float xs[4] = {keep[u].x, keep[u].y, keep[u].z, keep[u].w};
+      uint32_t word = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        word |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(xs[c], ts), __NV_SATFINITE, __NV_E4M3) << (8 * c);
+      reinterpret_cast<uint32_t *>(wcodes + went * D)[rank * L + lane] = word;
+      if (rank == 0 && lane == 0) wscales[went] = ts;
+    }
+  }
+  // no CTA leaves while another may still read its amaxima
   cl_sync();
 }
 
@@ -455,6 +505,35 @@ int launch_compress_ew(const float *x, const float *z, int B, int T, int D, int 
                        cudaStream_t stream) {
   const int L = D / 4;
   const int n = T / m;
+  if (m == kClGroups * kClUnroll && D % kClChannels == 0 && D / kClChannels <= 8 && n > 0) {
+    // large blocks: entries and window in one channel-split cluster pass
+    const int CG = D / kClChannels;
+    const int64_t grid = (int64_t)B * n * CG;
+    if (grid > 0x7fffffffLL) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_ew: too many entries");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, compress_cluster_kernel, x, z, n, D, m, x_bstride, codes, scales,
+                                             dst_first, dst_bstride, ring_cap, pooled, T, wcodes, wscales, w_first,
+                                             w_bstride, w_ring);
+    count_launches(1);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "compress_cluster_kernel launch: %s", cudaGetErrorString(e));
+    if (int rc = check_launch("compress_cluster_kernel")) return rc;
+    const int tail = T - n * m;                       // tokens past the last full block: window only
+    if (tail == 0) return CSA_OK;
+    const int64_t off = (int64_t)n * m * D;
+    return launch_compress(x + off, z + off, B, tail, D, 1, x_bstride, wcodes, wscales, w_first + (int64_t)n * m,
+                           w_bstride, w_ring, nullptr, stream);
+  }
   if ((m != 2 && m != 4 && m != 8) || L > kThreads || n == 0) {
     // not fused: the entries, then every token as a window entry
     if (int rc = launch_compress(x, z, B, T, D, m, x_bstride, codes, scales, dst_first, dst_bstride, ring_cap,
@@ -511,7 +590,8 @@ int launch_compress(const float *x, const float *z, int B, int T, int D, int m, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, compress_cluster_kernel, x, z, n, D, m, x_bstride, codes, scales,
-                                             dst_first, dst_bstride, ring_cap, pooled);
+                                             dst_first, dst_bstride, ring_cap, pooled, T, (uint8_t *)nullptr,
+                                             (float *)nullptr, (int64_t)0, (int64_t)0, 0);
     count_launches(1);
     if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "compress_cluster_kernel launch: %s", cudaGetErrorString(e));
     return check_launch("compress_cluster_kernel");

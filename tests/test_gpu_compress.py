@@ -151,3 +151,19 @@ def test_compress_ew_rings_and_offsets():
 def test_compress_ew_unfused_shapes(m):
     """m outside the fused range runs the two passes inside the call."""
     _ew_pair(2, 64, 512, m, cap=64 // m + 1, wcap=70, seed=m)
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 128 * 3 + 50, 512), (1, 256, 64), (3, 128, 256)])
+def test_compress_ew_m128_equals_two_passes(B, T, D):
+    """m' = 128 (the HCA block): entries and window in one channel-split
+    cluster pass, bit-identical to the two calls (including a ragged tail of
+    window-only tokens and the pooled output)."""
+    _ew_pair(B, T, D, 128, cap=T // 128 + 2, wcap=T + 3, seed=B + T, pooled=True)
+
+
+def test_compress_ew_m128_rings():
+    """The HCA append: one 128-token block per sequence at an entry offset,
+    its tokens into a window ring smaller than the call (only the last ring
+    slots' tokens survive) and an entry ring that wraps."""
+    _ew_pair(2, 128, 512, 128, cap=50, wcap=100, dst_first=40, win_first=7, win_ring=100, seed=11)
+    _ew_pair(2, 384, 512, 128, cap=2, wcap=128, dst_first=1, ring=2, win_first=0, win_ring=128, seed=12)
