@@ -32,14 +32,16 @@
 // N = 64 (about 50 cycles, its issue floor, against 135 at N = 256), so the
 // QK product runs at N = 64.
 //
-// Roles (288 threads):
-//   warps 0-3  gather 64 items per chunk (dense lists: one bulk L2 prefetch
-//              of the chunk two ahead), convert E4M3 codes exactly to bf16
-//              and store them in the "core matrix" layout (8 rows x 16 B);
-//   warps 4-7  first half of Q into TMEM, then softmax: one head per thread,
+// Roles (416 threads):
+//   warps 0-7  gather 64 items per chunk, one item row per thread and half
+//              of d (dense lists: one bulk L2 prefetch of the chunk two
+//              ahead), convert E4M3 codes exactly to bf16 and store them in
+//              the "core matrix" layout (8 rows x 16 B); with four warps the
+//              conversion and stores of a chunk (~2 us) paced the CTA;
+//   warps 8-11 first half of Q into TMEM, then softmax: one head per thread,
 //              lazy rescaling of O (only when a chunk raises the running max
 //              by more than 2^8), P = p * scale written to TMEM;
-//   warp 8     TMEM allocation, the Q TMA, and the single MMA-issuing thread,
+//   warp 12    TMEM allocation, the Q TMA, and the single MMA-issuing thread,
 //              which issues whichever of PV(c) and QK(c + 2) is ready first.
 // Item scales multiply the logits and P, never the codes, so the bf16 tiles
 // hold the E4M3 values exactly.  Every mbarrier wait is bounded by wall time;
@@ -55,7 +57,10 @@ constexpr int TD = 512;          // entry width
 constexpr int DHALF = 256;       // output columns per CTA = PV MMA N
 constexpr int CH = 64;           // items per chunk = QK MMA N
 constexpr uint32_t GS = CH * 16; // byte step between d-groups of a KV tile
-constexpr int kThreads = 288;
+constexpr int kLoadWarps = 8;    // warps 0-7 gather and convert the item tiles
+constexpr int kSoftWarp0 = 8;    // warps 8-11 run the softmax (TMEM lane quadrant = warp % 4)
+constexpr int kMmaWarp = 12;     // TMEM allocation, Q TMA, MMA issue
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kMaxSel = 2048;
 constexpr int kPrefetchAhead = 2;  // chunks
 constexpr float kLog2e = 1.4426950408889634f;
@@ -282,13 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
   if (tid == 0) {
     misc->abort = 0;
     for (int i = 0; i < kNumBars; ++i)
-      tc::mbar_init(&bars[i], (i < BAR_FREE_A || i == BAR_P_FULL || i == BAR_P_FULL + 1 || i == BAR_QT) ? 128 : 1);
+      tc::mbar_init(&bars[i], i < BAR_FREE_A ? 32 * kLoadWarps
+                                  : (i == BAR_P_FULL || i == BAR_P_FULL + 1 || i == BAR_QT) ? 128 : 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(&misc->tmem_base, TMEM_COLS);
-  } else if (SEL && a.idx) {
+  } else if (warp < 8 && SEL && a.idx) {
     // ordered compaction of the valid selected entries (warps 0-7)
     const int32_t *irow = a.idx + (int64_t)row * a.K;
     int base = 0;
@@ -333,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
     *scp = a.wscales + ent;
     return a.wcodes + ent * TD;
   };
-  if (warp == 8 && lane == 0 && nloc > 0) {
+  if (warp == kMmaWarp && lane == 0 && nloc > 0) {
     // second half of Q: 16 boxes of 128 heads x 16 d (32-byte swizzle, the
     // layout the MMA reads), box k = d 256 + 16 k
     tc::mbar_arrive_expect_tx(&bars[BAR_Q], TH * (TD / 2) * 2);
@@ -341,34 +347,29 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       tc::tma_load_2d(smem + OFF_QH + k * 4096, &qmap, TD / 2 + 16 * k, row * TH, &bars[BAR_Q]);
   }
 
-  if (warp < 4) {
+  if (warp < kLoadWarps) {
     // ------------------------------------------------------------ loaders
-    // 4 threads per item row; warp w takes items 32 r + 8 w + (0..7) of
-    // each chunk, thread (i8, pq) the 16-byte groups pq + 4 k of the row:
-    // k < 4 lie in d < 256, k >= 4 in d >= 256.  Half A (d outside this
-    // CTA's output half) first, half B after; each half's loads for the next
-    // chunk are issued as soon as the previous half is stored.
+    // 4 threads per item row; warp w takes items 8 w + (0..7) of each chunk,
+    // thread (i8, pq) the 16-byte groups pq + 4 k of the row: k < 4 lie in
+    // d < 256, k >= 4 in d >= 256.  Half A (d outside this CTA's output half)
+    // first, half B after; each half's loads for the next chunk are issued as
+    // soon as the previous half is stored.
     const int i8 = lane & 7, pq = lane >> 3;
+    const int item = warp * 8 + i8;
     const float qs = a.sm_scale * kLog2e;
     const int u_end = min(c_end * CH, n_items);
     const int ka = (1 - dh) * 4, kb = dh * 4;      // first k of half A / half B
-    uint4 ra[2][4], rb[2][4];
-    float sc[2];
-    auto load_half = [&](int lc, int k0, uint4 (&r)[2][4], bool with_scale) {
+    uint4 ra[4], rb[4];
+    float sc = 0.f;
+    auto load_half = [&](int lc, int k0, uint4 (&r)[4], bool with_scale) {
+      const int u = (c_begin + lc) * CH + item;
+      const float *scp;
+      const uint8_t *src = item_src(u, &scp);
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int item = i * 32 + warp * 8 + i8;
-        const int u = (c_begin + lc) * CH + item;
-        const float *scp;
-        const uint8_t *src = item_src(u, &scp);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) r[i][k] = __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * (k0 + k));
-        if (with_scale) {
-          // consumed only when the half is stored (items past the list get 0
-          // there), so the load's latency stays hidden
-          sc[i] = __ldg(scp);
-        }
-      }
+      for (int k = 0; k < 4; ++k) r[k] = __ldg(reinterpret_cast<const uint4 *>(src) + pq + 4 * (k0 + k));
+      // consumed only when the half is stored (items past the list get 0
+      // there), so the load's latency stays hidden
+      if (with_scale) sc = __ldg(scp);
       // dense lists: the entries of the chunk kPrefetchAhead ahead are
       // contiguous rows; one bulk prefetch pulls them into L2
       if (!SEL && with_scale && warp == 0 && lane == 0) {
@@ -379,18 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
                        ::"l"(a.codes + ((int64_t)b * a.entry_cap + f0) * TD), "r"((f1 - f0) * TD) : "memory");
       }
     };
-    auto store_half = [&](unsigned char *kv, int k0, const uint4 (&r)[2][4]) {
+    auto store_half = [&](unsigned char *kv, int k0, const uint4 (&r)[4]) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int item = i * 32 + warp * 8 + i8;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int p = pq + 4 * (k0 + k);
-          uint4 lo, hi;
-          e4m3x16_to_bf16x16(r[i][k], lo, hi);
-          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p)) = lo;
-          *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p + 1)) = hi;
-        }
+      for (int k = 0; k < 4; ++k) {
+        const int p = pq + 4 * (k0 + k);
+        uint4 lo, hi;
+        e4m3x16_to_bf16x16(r[k], lo, hi);
+        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p)) = lo;
+        *reinterpret_cast<uint4 *>(kv + kv_off(item, 2 * p + 1)) = hi;
       }
     };
     if (nloc > 0) {
@@ -409,22 +406,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       // half B and the item scales: free once PV(lc - 2) is done
       if (lc >= 2 && !wait_bar(&bars[BAR_FREE_B + kslot], ((lc - 2) >> 1) & 1, misc, a.status)) break;
       store_half(kv, kb, rb);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int item = i * 32 + warp * 8 + i8;
-        if (pq == 0) {
-          const float v = (c_begin + lc) * CH + item < n_items ? sc[i] : 0.f;
-          iscale[kslot * CH + item] = v;
-          lscale[kslot * CH + item] = v * qs;
-        }
+      if (pq == 0) {
+        const float v = (c_begin + lc) * CH + item < n_items ? sc : 0.f;
+        iscale[kslot * CH + item] = v;
+        lscale[kslot * CH + item] = v * qs;
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars[BAR_FULL_B + kslot]);
       if (lc + 1 < nloc) load_half(lc + 1, kb, rb, true);
     }
-  } else if (warp < 8) {
+  } else if (warp < kSoftWarp0 + 4) {
     // ------------------------------------------------------------ softmax
-    const int quad = warp - 4;
+    const int quad = warp - kSoftWarp0;
     const int h = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     bool ok = true;
@@ -639,6 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       // c & 1 read (PV(c - 2) issued); QK_B(c) needs half B; PV(c) needs P(c).
       // The first ready of PV, QK_B, QK_A goes next, so the tensor core works
       // on one chunk while the loaders and the softmax warps handle others.
+      // (Each product goes out whole: issuing QK in groups of 2-8 K steps, to
+      // let a ready PV in sooner, made the call 20-80 % slower.)
       const int half_a = 1 - dh, half_b = dh;
       int nqa = 0, nqb = 0, npv = 0;
       const uint64_t t0 = globaltimer();
@@ -709,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(const __grid_con
       }
     }
   }
-  if (warp == 8) tc::tmem_dealloc(tbase, TMEM_COLS);
+  if (warp == kMmaWarp) tc::tmem_dealloc(tbase, TMEM_COLS);
 }
 
 }  // namespace
