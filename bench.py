@@ -37,6 +37,10 @@ METRIC = "CSA/HCA decode tokens/s and prefill queries/s on 1 B200; % of HBM BW /
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# cycles of the device sleep that queues each separately timed call
+SLEEP_CYCLES = 2_000_000
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -483,12 +487,14 @@ def measure(args, wl, steps, world, rank, local, dev, peaks, peaks_src, cpu_budg
     ms_per_step = step_ms / steps
     value = job_throughput(world, r.units_per_step, ms_per_step)
 
-    # per-call device time: each call alone, cold L2, queued behind a bounded sleep
+    # per-call device time: each call alone, cold L2, queued behind a bounded
+    # sleep (~1 ms, longer than the binding's host-side launch work, so the
+    # events bracket device time only)
     per_call = {}
     for i in range(args.warmup, args.warmup + min(steps, 5)):
         for name, fn in r.calls(i):
             l2_flush(flush)
-            torch.cuda._sleep(200000)
+            torch.cuda._sleep(SLEEP_CYCLES)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record()
@@ -937,7 +943,7 @@ def kernel_case(args, wl):
     times = []
     for _ in range(args.steps):
         l2_flush(flush)
-        torch.cuda._sleep(200000)
+        torch.cuda._sleep(SLEEP_CYCLES)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
