@@ -103,6 +103,43 @@ def test_hca_attend_parity(B, Tq, H, D, m, N, W):
     parity.check_attention(out, lse, ro, rl)
 
 
+
+# The 128-head kernel splits each (row, half of D) into 1, 2, 4 or 8 item
+# splits, one thread-block cluster, from the row count and the longest item
+# list (splits * 2 * rows <= 148, at least two 64-item chunks per split); the
+# cases above all take 4.  These reach 8 (few rows, long lists; the last splits
+# of a row get no chunk at all), 2 and 1 (many rows), sparse and dense.
+SPLIT_CASES = [
+    # B, Tq, m, N, K, W, dense, splits the plan gives
+    (1, 1, 4, 1200, 1, 128, True, 8),     # 1,328 items = 21 chunks: 7 splits of 3, one empty
+    (1, 2, 4, 1500, 1024, 128, False, 8),  # 1,152 items = 18 chunks: 6 splits of 3, two empty
+    (2, 12, 4, 400, 64, 32, False, 2),     # 24 rows
+    (2, 20, 4, 300, 1, 32, True, 1),       # 40 rows
+]
+
+
+@pytest.mark.parametrize("B,Tq,m,N,K,W,dense,splits", SPLIT_CASES)
+def test_128_head_split_counts(B, Tq, m, N, K, W, dense, splits):
+    H, D = 128, 512
+    rng = np.random.default_rng(1000 + 10 * B + Tq)
+    if splits == 8:
+        # every row sees its whole list: the plan's longest list is reached
+        q_pos = (m * N - 1 - 37 * np.arange(B * Tq)).reshape(B, Tq).astype(np.int32)
+    else:
+        q_pos = rng.integers(0, m * N, (B, Tq)).astype(np.int32)
+        q_pos[0, 0] = 0
+        q_pos[-1, -1] = m * N - 1
+    codes, scales, wcodes, wscales, q, ent, wv = _setup(B, Tq, H, D, N, W, q_pos, 17, 512 ** -0.5)
+    d = Dims(B=B, Tq=Tq, H=H, D=D, K=K, W=W, m=m, n_entries=N, win_cap=W)
+    if dense:
+        out, lse = _run_gpu(q, codes, scales, None, wcodes, wscales, q_pos, d)
+        ro, rl = ocsa.hca_attend(_bits(q), ent, lambda b, p: wv[b, p % W], q_pos, m, W)
+    else:
+        idx = _random_selection(rng, q_pos, m, N, K)
+        out, lse = _run_gpu(q, codes, scales, idx, wcodes, wscales, q_pos, d)
+        ro, rl = ocsa.attend(_bits(q), ent, idx, lambda b, p: wv[b, p % W], q_pos, W)
+    parity.check_attention(out, lse, ro, rl)
+
 def test_softmax_scale_is_applied():
     B, Tq, H, D, m, N, K, W = 1, 3, 8, 64, 4, 50, 8, 16
     q_pos = np.array([[199, 100, 40]], dtype=np.int32)
