@@ -113,6 +113,16 @@ def test_small_k_and_window():
     _run_chain(4, 2000, 2, K=37, W=5, seed=9)
 
 
+
+@pytest.mark.parametrize("B", [1, 9, 37])
+def test_sequence_counts(B):
+    """One sequence (every SM scans a share of its keys; five attention splits
+    of one chunk per quarter of D), nine (16 scanning CTAs per sequence, three
+    splits of two chunks: the online softmax across chunks) and 37, the most
+    the step accepts (four scanning CTAs per sequence, one split of five
+    chunks per quarter, written without a merge)."""
+    _run_chain(B, 4096 if B == 1 else 2048, 3 if B == 1 else 2, seed=12 + B)
+
 def test_massive_ties_take_the_refinement():
     """Every indexer key equal: all scores tie, the threshold bin holds every
     entry and the exact tie refinement must pick the lowest indices."""
